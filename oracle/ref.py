@@ -1,0 +1,320 @@
+"""Float64 CPU oracle for exact scaled-dot-product attention.
+
+TEST INFRASTRUCTURE ONLY. This module is the slow, obviously-correct statement of
+what the GPU path computes. Only the test suite, the smoke check in
+``__graft_entry__`` and the ``cpu_baseline`` / reference arm of ``bench.py`` may
+import it. The product path (the CUDA library and its Python binding) never
+imports, calls or falls back to anything here, and nothing here imports the
+product path.
+
+Sources (web pages on FlashAttention, cited by title and section):
+
+* "Flash-Attention 2/3在ms-swift中的集成与性能提升" (FA2/3 in ms-swift), opening
+  formula: Attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V, and the statement that
+  the full score matrix S is what tiling avoids storing.
+* Qwen flash_attn explainer, section 一 "什么是 Attention": the three steps
+  (scores Q.K^T, scale by 1/sqrt(d_k) and softmax, weighted sum of V).
+* "FlashAttention优化Transformer显存与计算效率", section 2.1 (the naive
+  computation over [batch, heads, seq_len, dim]) and section 2.2.2 (blockwise
+  softmax: per block a max m and an exp-sum l, combined stably).
+* "突破AI算力瓶颈：FlashAttention与MindSpore 2.0全场景融合方案", section
+  推理优化与KV缓存 (flash_attn_with_kvcache: append one K/V row per step at
+  position cache_seqlens, attend one query row, causal=True).
+
+Readings taken where the pages are silent (each is also listed in the design notes):
+
+* Layout: tensors are [B, N, H, d] (batch, seq_len, heads, head_dim), as in the
+  ms-swift long-text page section 1.1.
+* scale=None means 1/sqrt(d) (the formula's d_k).
+* LSE is the natural-log log-sum-exp of the *scaled* scores of each query row
+  over its visible keys, laid out [B, H, Nq].
+* Causal with Nq != Nk aligns bottom-right: key j is visible to query i iff
+  j <= i + (Nk - Nq). With Nq == Nk this is the usual j <= i.
+* A query row with no visible key returns out = 0 and lse = -inf.
+* cache_seqlens[b] is the number of valid cache rows before the step's append;
+  with k_new given, the new row is written at that index and attention covers
+  cache_seqlens[b] + 1 rows; without it, it covers cache_seqlens[b] rows.
+* The backward is the analytic gradient of the definition (the pages only say the
+  scores are recomputed, not stored).
+
+Every array is numpy float64; callers convert the exact bf16 input values first.
+Large problems are processed in blocks of query rows; each block's softmax is the
+exact row softmax over all keys (no online rescaling), so blocking does not change
+the arithmetic beyond floating-point summation order inside BLAS.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "default_scale",
+    "visible_mask",
+    "scores",
+    "softmax_rows",
+    "attention_forward",
+    "attention_backward",
+    "blockwise_forward",
+    "merge_partials",
+    "decode_step",
+    "decode_sequence",
+]
+
+
+def default_scale(d: int) -> float:
+    """softmax_scale=None -> 1/sqrt(d_k) (the formula of the ms-swift FA2/3 page)."""
+    return 1.0 / math.sqrt(d)
+
+
+def visible_mask(q_pos: np.ndarray, nk: int, causal: bool, nq_total: int) -> np.ndarray:
+    """Boolean [len(q_pos), nk] mask of keys each query may attend to.
+
+    Causal uses bottom-right alignment: key j visible to query i iff
+    j <= i + (nk - nq_total). Non-causal sees every key.
+    """
+    j = np.arange(nk)[None, :]
+    if not causal:
+        return np.ones((len(q_pos), nk), dtype=bool)
+    return j <= (np.asarray(q_pos)[:, None] + (nk - nq_total))
+
+
+def scores(qm: np.ndarray, km: np.ndarray, scale: float) -> np.ndarray:
+    """S = scale * Q K^T for one (batch, head): [nq, d] x [nk, d] -> [nq, nk]."""
+    return scale * (qm @ km.T)
+
+
+def softmax_rows(s: np.ndarray, mask: np.ndarray):
+    """Max-subtracted row softmax with masked entries excluded.
+
+    Returns (P, lse). Rows with no visible entry give P = 0 and lse = -inf.
+    """
+    s = np.where(mask, s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    e = np.where(mask, np.exp(s - m_safe), 0.0)
+    l = np.sum(e, axis=1, keepdims=True)
+    p = np.where(empty, 0.0, e / np.where(empty, 1.0, l))
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, m_safe + np.log(np.where(empty, 1.0, l)))
+    return p, lse[:, 0]
+
+
+def _resolve_scale(scale, d):
+    return default_scale(d) if scale is None else float(scale)
+
+
+def attention_forward(q, k, v, causal=False, scale=None, row_block=1024,
+                      heads=None, rows=None):
+    """Exact attention forward, materialising S per (b, h) in query-row blocks.
+
+    q: [B, Nq, H, d]; k, v: [B, Nk, H, d] (float64).
+    Returns out [B, Nq, H, d] and lse [B, H, Nq].
+
+    ``heads`` (list of (b, h)) and ``rows`` (sorted query indices) restrict the
+    work to a sample; entries outside the sample are left as NaN.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    sc = _resolve_scale(scale, d)
+    out = np.full((B, Nq, H, v.shape[3]), np.nan)
+    lse = np.full((B, H, Nq), np.nan)
+    head_list = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    row_idx = np.arange(Nq) if rows is None else np.asarray(rows)
+    for (b, h) in head_list:
+        km = k[b, :, h, :]
+        vm = v[b, :, h, :]
+        for s0 in range(0, len(row_idx), row_block):
+            ridx = row_idx[s0:s0 + row_block]
+            qm = q[b, ridx, h, :]
+            mask = visible_mask(ridx, Nk, causal, Nq)
+            p, l = softmax_rows(scores(qm, km, sc), mask)
+            out[b, ridx, h, :] = p @ vm
+            lse[b, h, ridx] = l
+    return out, lse
+
+
+def attention_backward(q, k, v, dout, causal=False, scale=None, row_block=1024,
+                       heads=None):
+    """Analytic gradients of out = softmax(scale*Q K^T, mask) V.
+
+    With P the row softmax and dO the output gradient:
+      dV = P^T dO,  dP = dO V^T,  dS = P * (dP - rowsum(P * dP)),
+      dQ = scale * dS K,  dK = scale * dS^T Q.
+    S is rebuilt from Q and K in query-row blocks (recomputation, as the pages
+    describe for the backward pass), never stored whole.
+    Returns dq, dk, dv with the shapes of q, k, v (NaN outside ``heads``).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    sc = _resolve_scale(scale, d)
+    dq = np.full(q.shape, np.nan)
+    dk = np.full(k.shape, np.nan)
+    dv = np.full(v.shape, np.nan)
+    head_list = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    for (b, h) in head_list:
+        km = k[b, :, h, :]
+        vm = v[b, :, h, :]
+        dk_acc = np.zeros((Nk, d))
+        dv_acc = np.zeros((Nk, v.shape[3]))
+        for r0 in range(0, Nq, row_block):
+            ridx = np.arange(r0, min(Nq, r0 + row_block))
+            qm = q[b, ridx, h, :]
+            dom = dout[b, ridx, h, :]
+            mask = visible_mask(ridx, Nk, causal, Nq)
+            p, _ = softmax_rows(scores(qm, km, sc), mask)
+            dv_acc += p.T @ dom
+            dp = dom @ vm.T
+            rowdot = np.sum(p * dp, axis=1, keepdims=True)
+            ds = p * (dp - rowdot)
+            dq[b, ridx, h, :] = sc * (ds @ km)
+            dk_acc += sc * (ds.T @ qm)
+        dk[b, :, h, :] = dk_acc
+        dv[b, :, h, :] = dv_acc
+    return dq, dk, dv
+
+
+def merge_partials(o_parts, lse_parts):
+    """Combine partial attention results computed over disjoint key sets.
+
+    Each part s holds o_s (its own normalised output) and lse_s (its own
+    log-sum-exp). This is the stable combination of the per-block max m and
+    exp-sum l described in section 2.2.2 of "FlashAttention优化Transformer显存与
+    计算效率", written in log space: LSE = log sum_s exp(lse_s) and
+    O = sum_s exp(lse_s - LSE) o_s. Parts with lse_s = -inf contribute nothing.
+
+    o_parts: [S, ..., d]; lse_parts: [S, ...]. Returns (o, lse).
+    """
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = np.max(lse_parts, axis=0)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    w = np.exp(lse_parts - m_safe[None])
+    tot = np.sum(w, axis=0)
+    with np.errstate(divide="ignore"):
+        lse = np.where(empty, -np.inf, m_safe + np.log(np.where(empty, 1.0, tot)))
+    coef = np.where(empty[None], 0.0, w / np.where(empty, 1.0, tot)[None])
+    o = np.sum(coef[..., None] * o_parts, axis=0)
+    return o, lse
+
+
+def blockwise_forward(q, k, v, causal=False, scale=None, block_q=64, block_k=64):
+    """Tiled forward with a running max m and running sum l per query row.
+
+    Restates section 2.2.1/2.2.2 of "FlashAttention优化Transformer显存与计算效率":
+    loop over query blocks and, inside, over key blocks; for each key block take
+    the block's row max and exp-sum and fold them into the running (m, l, acc)
+    with the rescale factor exp(m_old - m_new). The full S is never formed. Used
+    only to check the materialising oracle above.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    sc = _resolve_scale(scale, d)
+    out = np.zeros((B, Nq, H, v.shape[3]))
+    lse = np.zeros((B, H, Nq))
+    for b in range(B):
+        for h in range(H):
+            for i0 in range(0, Nq, block_q):
+                ridx = np.arange(i0, min(Nq, i0 + block_q))
+                qb = q[b, ridx, h, :]
+                m = np.full(len(ridx), -np.inf)
+                l = np.zeros(len(ridx))
+                acc = np.zeros((len(ridx), v.shape[3]))
+                for j0 in range(0, Nk, block_k):
+                    cidx = np.arange(j0, min(Nk, j0 + block_k))
+                    s = sc * (qb @ k[b, cidx, h, :].T)
+                    vis = visible_mask(ridx, Nk, causal, Nq)[:, cidx]
+                    s = np.where(vis, s, -np.inf)
+                    m_blk = np.max(s, axis=1)
+                    m_new = np.maximum(m, m_blk)
+                    base = np.where(np.isfinite(m_new), m_new, 0.0)
+                    alpha = np.where(np.isfinite(m), np.exp(m - base), 0.0)
+                    p = np.where(vis, np.exp(s - base[:, None]), 0.0)
+                    l = alpha * l + np.sum(p, axis=1)
+                    acc = alpha[:, None] * acc + p @ v[b, cidx, h, :]
+                    m = m_new
+                empty = l == 0.0
+                out[b, ridx, h, :] = np.where(empty[:, None], 0.0,
+                                              acc / np.where(empty, 1.0, l)[:, None])
+                with np.errstate(divide="ignore"):
+                    lse[b, h, ridx] = np.where(empty, -np.inf,
+                                               np.where(np.isfinite(m), m, 0.0)
+                                               + np.log(np.where(empty, 1.0, l)))
+    return out, lse
+
+
+def decode_step(q, k_cache, v_cache, cache_seqlens, k_new=None, v_new=None,
+                scale=None):
+    """One incremental decode step (flash_attn_with_kvcache, MindSpore page,
+    section 推理优化与KV缓存).
+
+    q: [B, 1, H, d]; caches: [B, Ncap, H, d]; cache_seqlens: int [B] = valid rows
+    before this step. With k_new/v_new ([B, 1, H, d]) the new row is written at
+    index cache_seqlens[b] of *copies* of the caches and the query attends rows
+    [0, cache_seqlens[b] + 1); without them it attends rows [0, cache_seqlens[b]).
+    A single query row at the end of the sequence sees every valid key, so the
+    causal flag changes nothing here (bottom-right alignment).
+
+    Returns (out [B, 1, H, d], lse [B, H], k_cache', v_cache').
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kc = np.array(k_cache, dtype=np.float64, copy=True)
+    vc = np.array(v_cache, dtype=np.float64, copy=True)
+    B, _, H, d = q.shape
+    Ncap = kc.shape[1]
+    sc = _resolve_scale(scale, d)
+    out = np.zeros((B, 1, H, vc.shape[3]))
+    lse = np.zeros((B, H))
+    for b in range(B):
+        L = int(cache_seqlens[b])
+        if k_new is not None:
+            if L + 1 > Ncap:
+                raise ValueError("cache full: cache_seqlens[b] + 1 > capacity")
+            kc[b, L] = np.asarray(k_new, dtype=np.float64)[b, 0]
+            vc[b, L] = np.asarray(v_new, dtype=np.float64)[b, 0]
+            L += 1
+        if L > Ncap:
+            raise ValueError("cache_seqlens[b] > capacity")
+        for h in range(H):
+            if L == 0:
+                out[b, 0, h] = 0.0
+                lse[b, h] = -np.inf
+                continue
+            s = scores(q[b, :, h, :], kc[b, :L, h, :], sc)
+            p, l = softmax_rows(s, np.ones_like(s, dtype=bool))
+            out[b, 0, h] = (p @ vc[b, :L, h, :])[0]
+            lse[b, h] = l[0]
+    return out, lse, kc, vc
+
+
+def decode_sequence(q_steps, k_steps, v_steps, k_cache, v_cache, start_seqlens,
+                    scale=None):
+    """Replay T decode steps with append (the incremental loop of the MindSpore
+    page): step t uses cache_seqlens = start_seqlens + t.
+
+    q_steps, k_steps, v_steps: [T, B, 1, H, d]. Returns outs [T, B, 1, H, d],
+    lses [T, B, H] and the final caches.
+    """
+    kc = np.asarray(k_cache, dtype=np.float64)
+    vc = np.asarray(v_cache, dtype=np.float64)
+    T = len(q_steps)
+    outs, lses = [], []
+    seq = np.asarray(start_seqlens, dtype=np.int64)
+    for t in range(T):
+        o, l, kc, vc = decode_step(q_steps[t], kc, vc, seq + t, k_steps[t], v_steps[t],
+                                   scale=scale)
+        outs.append(o)
+        lses.append(l)
+    return np.stack(outs), np.stack(lses), kc, vc
