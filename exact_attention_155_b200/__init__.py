@@ -1,0 +1,12 @@
+"""B200 (sm_100a) exact attention: fused forward with LSE, recompute backward and
+KV-cache decode, exposed through the C ABI of libfa.so (include/fa.h).
+
+The CUDA library is loaded lazily on the first call, so importing the package (for
+example for its seeded input generators) needs no GPU. Calls raise if the library
+is missing or the device is not sm_100.
+"""
+from .ops import (FAError, bwd, bwd_workspace_size, decode, decode_workspace_size,  # noqa: F401
+                  device_status, fwd, load_library)
+
+__all__ = ["FAError", "fwd", "bwd", "decode", "bwd_workspace_size", "decode_workspace_size",
+           "device_status", "load_library"]

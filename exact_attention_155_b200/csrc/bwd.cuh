@@ -1,0 +1,487 @@
+// Attention backward for sm_100a with recomputation: the score matrix is rebuilt
+// from Q, K and the forward's LSE tile by tile instead of being stored (the
+// "重计算 / Recomputation" item of the ms-swift FA2/3 page and of section 三 of the
+// Qwen flash_attn explainer). The gradient formulas are the analytic derivative of
+// softmax(scale Q K^T) V:
+//   P = exp(scale S - LSE), dV = P^T dO, dP = dO V^T, D_i = sum_c dO_ic O_ic,
+//   dS = P * (dP - D), dK = scale dS^T Q, dQ = scale dS K.
+//
+// Kernels:
+//  * bwd_pre_kernel: D per query row, the LSE converted to log2 units, zeroed fp32
+//    dQ accumulator. Rows are padded to a multiple of 128 (LSE = +inf there, so the
+//    recomputed P of a padded row is exactly 0).
+//  * bwd_kernel: one CTA per (batch, head, 128-key tile). K_j and V_j stay in shared
+//    memory; the CTA walks the query tiles i (i >= j when causal). Scores are
+//    computed transposed (keys on TMEM lanes) so P^T and dS^T are already in the
+//    A-operand orientation of dV += P^T dO and dK += dS^T Q:
+//       S^T  = K Q_i^T        (TMEM cols [0,128), fp32; P^T bf16 over [0,64))
+//       dP^T = V dO_i^T       (TMEM cols [128,256), fp32)
+//       dV  += P^T dO_i       (A from TMEM, TMEM cols [256,256+d))
+//       dK  += dS^T Q_i       (A = dS^T in shared memory, TMEM [256+d,256+2d))
+//       dQ_i = dS K           (A = the same shared buffer read MN-major,
+//                              TMEM cols [128,128+d) once dP^T has been read)
+//    Warps 0-3 (one key row per thread) turn S^T into P^T and dP^T into dS^T;
+//    warps 4-7 (one query row per thread) drain dQ_i from TMEM into the fp32
+//    accumulator with vector atomics; warp 8 issues TMA; warp 9 issues tcgen05.mma.
+//  * bwd_dq_convert_kernel: dq = bf16(accumulator).
+#pragma once
+
+#include <math.h>
+
+#include "ptx.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  int B, H, N, Np;      // Np = N rounded up to a multiple of 128
+  int nqt;              // Np / 128
+  float scale;          // softmax scale
+  float scale_log2;     // scale * log2(e)
+  const uint16_t* out;  // forward output [B, N, H, d]
+  const uint16_t* dout; // [B, N, H, d]
+  const float* lse;     // [B, H, N] natural log
+  float* dq_acc;        // [B, H, Np, d] fp32
+  float* lse2;          // [B, H, Np] log2 units (+inf on padded rows)
+  float* dvec;          // [B, H, Np] rowsum(dO * O)
+  uint16_t* dq;         // [B, N, H, d]
+  uint16_t* dk;
+  uint16_t* dv;
+};
+
+struct BwdWorkspace {
+  size_t dq_off, lse2_off, dvec_off, total;
+};
+
+inline size_t round256(size_t x) { return (x + 255) / 256 * 256; }
+
+inline BwdWorkspace bwd_ws_layout(int B, int H, int N, int d) {
+  const size_t Np = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t rows = static_cast<size_t>(B) * H * Np;
+  BwdWorkspace w;
+  w.dq_off = 0;
+  w.lse2_off = round256(rows * d * sizeof(float));
+  w.dvec_off = w.lse2_off + round256(rows * sizeof(float));
+  w.total = w.dvec_off + round256(rows * sizeof(float));
+  return w;
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
+  constexpr int TPR = D / 8;  // threads per row, 16 bytes each
+  const long long gt = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  const long long total = static_cast<long long>(p.B) * p.H * p.Np;
+  const long long row = gt / TPR;
+  const int sub = static_cast<int>(gt % TPR);
+  const bool valid = row < total;
+  const int i = valid ? static_cast<int>(row % p.Np) : 0;
+  const long long bh = valid ? row / p.Np : 0;
+  const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
+  float acc = 0.f;
+  if (valid && i < p.N) {
+    const size_t off = ((static_cast<size_t>(b) * p.N + i) * p.H + h) * D + sub * 8;
+    const uint4 o = __ldg(reinterpret_cast<const uint4*>(p.out + off));
+    const uint4 g = __ldg(reinterpret_cast<const uint4*>(p.dout + off));
+    const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc = fmaf(__uint_as_float(ow[k] << 16), __uint_as_float(gw[k] << 16), acc);
+      acc = fmaf(__uint_as_float(ow[k] & 0xFFFF0000u), __uint_as_float(gw[k] & 0xFFFF0000u), acc);
+    }
+  }
+#pragma unroll
+  for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (!valid) return;
+  if (sub == 0) {
+    const bool real = i < p.N;
+    p.dvec[row] = real ? acc : 0.f;
+    p.lse2[row] = real ? p.lse[bh * p.N + i] * 1.4426950408889634f : INFINITY;
+  }
+  float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D + sub * 8);
+  z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+  z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const BwdParams p) {
+  constexpr int TPR = D / 8;
+  const long long gt = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  const long long total = static_cast<long long>(p.B) * p.N * p.H;
+  const long long row = gt / TPR;  // (b, i, h) in output order
+  if (row >= total) return;
+  const int sub = static_cast<int>(gt % TPR);
+  const int h = static_cast<int>(row % p.H);
+  const long long bi = row / p.H;
+  const int i = static_cast<int>(bi % p.N);
+  const int b = static_cast<int>(bi / p.N);
+  const float4* src = reinterpret_cast<const float4*>(
+      p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * p.Np + i) * D + sub * 8);
+  const float4 a = src[0], c = src[1];
+  uint4 o;
+  o.x = pack_bf16x2(a.x, a.y);
+  o.y = pack_bf16x2(a.z, a.w);
+  o.z = pack_bf16x2(c.x, c.y);
+  o.w = pack_bf16x2(c.z, c.w);
+  *reinterpret_cast<uint4*>(p.dq + row * D + sub * 8) = o;
+}
+
+template <int D>
+struct BwdLayout {
+  static constexpr int kTile = 128 * D * 2;  // one 128-row bf16 tile
+  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr int kK = 0;
+  static constexpr int kV = kTile;
+  static constexpr int kStage0 = 2 * kTile;  // stage s: Q at +0, dO at +kTile
+  static constexpr int kStageBytes = 2 * kTile;
+  static constexpr int kDS = kStage0 + kStages * kStageBytes;  // 128 x 128 bf16 dS^T
+  static constexpr int kVec = kDS + 32768;                     // per stage: lse2[128], D[128]
+  static constexpr int kBar = kVec + kStages * 1024;
+  static constexpr int kKVFull = 0;
+  static constexpr int kStFull = 1;                  // [kStages]
+  static constexpr int kStEmpty = 1 + kStages;       // [kStages]
+  static constexpr int kSFull = 1 + 2 * kStages;
+  static constexpr int kDPFull = kSFull + 1;
+  static constexpr int kPFull = kSFull + 2;
+  static constexpr int kDSFull = kSFull + 3;
+  static constexpr int kDSFree = kSFull + 4;
+  static constexpr int kDQFull = kSFull + 5;
+  static constexpr int kDQFree = kSFull + 6;
+  static constexpr int kMmaDone = kSFull + 7;
+  static constexpr int kDrain = kSFull + 8;
+  static constexpr int kNumBars = kDrain + 1;
+  static constexpr int kMisc = kBar + kNumBars * 8;
+  static constexpr int kBytes = kMisc + 16;
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+enum : unsigned int {
+  kSiteBwdProducer = 0x201,
+  kSiteBwdMma = 0x202,
+  kSiteBwdSoftmax = 0x203,
+  kSiteBwdDrain = 0x204,
+  kSiteBwdSmemAlign = 0x2FF
+};
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c),
+               "f"(d)
+               : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1)
+    bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+               const BwdParams p) {
+  using L = BwdLayout<D>;
+  extern __shared__ __align__(1024) uint8_t smem[];
+  const uint32_t base = smem_u32(smem);
+  if (base & 1023u) {
+    // The swizzled tiles need a 1024-byte aligned base; there is no slack to realign.
+    if (threadIdx.x == 0) report(kDevTimeout, kSiteBwdSmemAlign, base);
+    return;
+  }
+  const uint32_t sK = base + L::kK, sV = base + L::kV, sDS = base + L::kDS;
+  const uint32_t bar0 = base + L::kBar;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMisc + 4);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+  const int warp = warp_id(), lane = lane_id();
+  const int BH = p.B * p.H;
+  const int jt = static_cast<int>(blockIdx.x) / BH;  // key tile; low ids = most work when causal
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.H, h = bh % p.H;
+  const int it0 = CAUSAL ? jt : 0;
+  const int niter = p.nqt - it0;
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(L::kKVFull), 1);
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(BAR(L::kStFull + s), 1);
+      mbar_init(BAR(L::kStEmpty + s), 1);
+    }
+    mbar_init(BAR(L::kSFull), 1);
+    mbar_init(BAR(L::kDPFull), 1);
+    mbar_init(BAR(L::kPFull), 128);
+    mbar_init(BAR(L::kDSFull), 128);
+    mbar_init(BAR(L::kDSFree), 1);
+    mbar_init(BAR(L::kDQFull), 1);
+    mbar_init(BAR(L::kDQFree), 128);
+    mbar_init(BAR(L::kMmaDone), 1);
+    mbar_init(BAR(L::kDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 128, tDV = tmem + 256,
+                 tDK = tmem + 256 + D;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(BAR(L::kKVFull), 2 * L::kTile);
+      for (int bx = 0; bx < D / 64; ++bx) {
+        tma_load_4d(sK + bx * 16384, &tmK, BAR(L::kKVFull), bx * 64, h, jt * 128, b);
+        tma_load_4d(sV + bx * 16384, &tmV, BAR(L::kKVFull), bx * 64, h, jt * 128, b);
+      }
+      const float* lse2_h = p.lse2 + static_cast<size_t>(bh) * p.Np;
+      const float* dvec_h = p.dvec + static_cast<size_t>(bh) * p.Np;
+      int n = 0;
+      for (; n < niter; ++n) {
+        const int it = it0 + n;
+        const int s = n % L::kStages;
+        if (!wait_bar(BAR(L::kStEmpty + s), ((n / L::kStages) & 1) ^ 1u, abort_flag, kSiteBwdProducer))
+          break;
+        const uint32_t st = base + L::kStage0 + s * L::kStageBytes;
+        mbar_arrive_expect_tx(BAR(L::kStFull + s), 2 * L::kTile + 1024);
+        for (int bx = 0; bx < D / 64; ++bx) {
+          tma_load_4d(st + bx * 16384, &tmQ, BAR(L::kStFull + s), bx * 64, h, it * 128, b);
+          tma_load_4d(st + L::kTile + bx * 16384, &tmdO, BAR(L::kStFull + s), bx * 64, h, it * 128, b);
+        }
+        const uint32_t sv = base + L::kVec + s * 1024;
+        bulk_load(sv, lse2_h + it * 128, 512, BAR(L::kStFull + s));
+        bulk_load(sv + 512, dvec_h + it * 128, 512, BAR(L::kStFull + s));
+      }
+      for (int k = max(0, n - L::kStages); k < n; ++k)
+        drain_wait(BAR(L::kStFull + k % L::kStages), (k / L::kStages) & 1);
+      drain_wait(BAR(L::kKVFull), 0);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
+      constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, 0, 1);   // dV (A in TMEM), dK (A K-major)
+      constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, 1, 1);    // dQ (A MN-major)
+      bool ok = wait_bar(BAR(L::kKVFull), 0, abort_flag, kSiteBwdMma);
+      for (int n = 0; n < niter && ok; ++n) {
+        const int s = n % L::kStages;
+        const uint32_t sQ = base + L::kStage0 + s * L::kStageBytes;
+        const uint32_t sdO = sQ + L::kTile;
+        if (!(ok = wait_bar(BAR(L::kStFull + s), (n / L::kStages) & 1, abort_flag, kSiteBwdMma))) break;
+        tc_fence_after();
+        // S^T = K Q_i^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
+          umma_ss(tS, sdesc_sw128(sK + koff, 16, 1024), sdesc_sw128(sQ + koff, 16, 1024), kIdS,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(BAR(L::kSFull));
+        // dP^T = V dO_i^T into the region dQ_{i-1} used: wait until it was drained.
+        if (n > 0) {
+          if (!(ok = wait_bar(BAR(L::kDQFree), (n - 1) & 1, abort_flag, kSiteBwdMma))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
+          umma_ss(tDP, sdesc_sw128(sV + koff, 16, 1024), sdesc_sw128(sdO + koff, 16, 1024), kIdS,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(BAR(L::kDPFull));
+        // dV += P^T dO_i
+        if (!(ok = wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
+                  (n > 0 || kk > 0) ? 1u : 0u);
+        // dK += dS^T Q_i ; dQ_i = dS K
+        if (!(ok = wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tDK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+                  sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdKV, (n > 0 || kk > 0) ? 1u : 0u);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tDQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                  sdesc_sw128(sK + kk * 2048, 16384, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        umma_commit(BAR(L::kDQFull));
+        umma_commit(BAR(L::kDSFree));
+        umma_commit(BAR(L::kStEmpty + s));
+      }
+      if (ok) umma_commit(BAR(L::kMmaDone));
+      umma_commit(BAR(L::kDrain));
+      drain_wait(BAR(L::kDrain), 0);
+    }
+  } else if (warp < 4) {
+    // -------------------------------------------- P^T and dS^T (one key per thread)
+    const int r = warp * 32 + lane;
+    const int key = jt * 128 + r;
+    const bool key_ok = key < p.N;
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int n = 0; n < niter; ++n) {
+      const int it = it0 + n;
+      const int s = n % L::kStages;
+      const float* vec = reinterpret_cast<const float*>(smem + L::kVec + s * 1024);
+      ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kSFull), n & 1, abort_flag, kSiteBwdSoftmax));
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kStFull + s), (n / L::kStages) & 1,
+                                                   abort_flag, kSiteBwdSoftmax));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32(tS + lane_off + 0, s0);
+      tmem_ld32(tS + lane_off + 32, s1);
+      tmem_ld32(tS + lane_off + 64, s2);
+      tmem_ld32(tS + lane_off + 96, s3);
+      tmem_wait_ld();
+      reg_fence32(s0);
+      reg_fence32(s1);
+      reg_fence32(s2);
+      reg_fence32(s3);
+      // Queries of this tile that key `key` may not attend: q < key (causal) or key >= N.
+      const int qlim = !key_ok ? 1 << 30 : (CAUSAL ? key - it * 128 : 0);
+      uint32_t pk[64];
+#pragma unroll
+      for (int c2 = 0; c2 < 64; ++c2) {
+        const int c = 2 * c2;
+        const uint32_t* src = c < 32 ? s0 : (c < 64 ? s1 : (c < 96 ? s2 : s3));
+        const float x0 = __uint_as_float(src[c & 31]) * sl2 - vec[c];
+        const float x1 = __uint_as_float(src[(c + 1) & 31]) * sl2 - vec[c + 1];
+        const float p0 = (c < qlim) ? 0.f : ex2_approx(x0);
+        const float p1 = (c + 1 < qlim) ? 0.f : ex2_approx(x1);
+        pk[c2] = pack_bf16x2(p0, p1);
+      }
+      {
+        uint32_t a[32], bq[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          a[c] = pk[c];
+          bq[c] = pk[32 + c];
+        }
+        tmem_st32(tS + lane_off + 0, a);
+        tmem_st32(tS + lane_off + 32, bq);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(L::kPFull));
+
+      ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDPFull), n & 1, abort_flag, kSiteBwdSoftmax));
+      if (ok && n > 0)
+        ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDSFree), (n - 1) & 1, abort_flag, kSiteBwdSoftmax));
+      if (!ok) break;
+      tc_fence_after();
+      const float* dvec = vec + 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t dp[32];
+        tmem_ld32(tDP + lane_off + q * 32, dp);
+        tmem_wait_ld();
+        reg_fence32(dp);
+        uint32_t w[16];
+#pragma unroll
+        for (int c2 = 0; c2 < 16; ++c2) {
+          const uint32_t pp = pk[q * 16 + c2];
+          const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xFFFF0000u);
+          const int c = q * 32 + 2 * c2;
+          const float d0 = p0 * (__uint_as_float(dp[2 * c2]) - dvec[c]);
+          const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1]) - dvec[c + 1]);
+          w[c2] = pack_bf16x2(d0, d1);
+        }
+        // Row r of the dS^T tile, queries q*32 .. q*32+31, 128-byte swizzle.
+        const uint32_t row_base = sDS + (q >> 1) * 16384 + r * 128;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = (q & 1) * 4 + ch;
+          st_shared_v4(row_base + ((chunk ^ (r & 7)) << 4), w[4 * ch], w[4 * ch + 1], w[4 * ch + 2],
+                       w[4 * ch + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(BAR(L::kDSFull));
+    }
+    if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kMmaDone), 0, abort_flag, kSiteBwdSoftmax));
+    if (ok) {
+      tc_fence_after();
+      const size_t orow = ((static_cast<size_t>(b) * p.N + key) * p.H + h) * D;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tsrc = (which == 0 ? tDV : tDK) + lane_off;
+        const float mul = which == 0 ? 1.f : p.scale;
+        uint16_t* dst = (which == 0 ? p.dv : p.dk) + orow;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tsrc + cc * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+          if (key_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              d4[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * mul, __uint_as_float(o[8 * v + 1]) * mul),
+                                 pack_bf16x2(__uint_as_float(o[8 * v + 2]) * mul, __uint_as_float(o[8 * v + 3]) * mul),
+                                 pack_bf16x2(__uint_as_float(o[8 * v + 4]) * mul, __uint_as_float(o[8 * v + 5]) * mul),
+                                 pack_bf16x2(__uint_as_float(o[8 * v + 6]) * mul, __uint_as_float(o[8 * v + 7]) * mul));
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------- dQ drain (one query per thread)
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    for (int n = 0; n < niter; ++n) {
+      const int it = it0 + n;
+      const bool ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDQFull), n & 1, abort_flag, kSiteBwdDrain));
+      if (!ok) break;
+      tc_fence_after();
+      const int qrow = it * 128 + r;
+      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Np + qrow) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tDQ + lane_off + cc * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        if (qrow < p.N) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            red_add_v4(dst + cc * 32 + 4 * v, __uint_as_float(o[4 * v]) * p.scale,
+                       __uint_as_float(o[4 * v + 1]) * p.scale, __uint_as_float(o[4 * v + 2]) * p.scale,
+                       __uint_as_float(o[4 * v + 3]) * p.scale);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(BAR(L::kDQFree));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+#undef BAR
+}
+
+}  // namespace fa

@@ -1,0 +1,449 @@
+// C ABI of libfa.so: argument checking, TMA descriptor encoding and kernel launch.
+// Declarations and the contract of every entry point are in include/fa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+#include <set>
+#include <utility>
+#include <string>
+
+#include "fa.h"
+#include "ptx.cuh"
+#include "fwd.cuh"
+#include "bwd.cuh"
+#include "decode.cuh"
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+thread_local std::string g_last_error;
+
+fa_status fail(fa_status st, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+fa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(FA_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+// ---------------------------------------------------------------- device info
+struct DeviceInfo {
+  bool queried = false;
+  bool supported = false;
+  int sms = 0;
+  std::string why;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+fa_status current_device(int* dev_out, int* sms_out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(FA_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.queried) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    di.queried = true;
+    di.sms = sms;
+    di.supported = (major == 10 && minor == 0);
+    if (!di.supported) {
+      char buf[128];
+      snprintf(buf, sizeof(buf), "device %d is sm_%d%d; this library is built for sm_100a only", dev,
+               major, minor);
+      di.why = buf;
+    }
+  }
+  if (!di.supported) return fail(FA_ERR_UNSUPPORTED, "%s", di.why.c_str());
+  if (dev_out) *dev_out = dev;
+  if (sms_out) *sms_out = di.sms;
+  return FA_OK;
+}
+
+// SM count used for sizing decisions that must also be answerable without a GPU
+// (workspace queries): the current device's count when there is one, else 148.
+int sm_count_or_default() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess &&
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
+    return sms;
+  cudaGetLastError();  // clear the "no device" error so it does not leak into later calls
+  return 148;
+}
+
+// ------------------------------------------------------------- TMA descriptors
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+fa_status get_encoder(EncodeTiledFn* fn) {
+  static EncodeTiledFn cached = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) cached = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!cached) {
+    if (err != cudaSuccess) return cuda_fail(err, "cudaGetDriverEntryPoint(cuTensorMapEncodeTiled)");
+    return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  }
+  *fn = cached;
+  return FA_OK;
+}
+
+// 4-D map over a [B, N, H, d] bf16 tensor; one box = 128 rows of one (b, h) x 64
+// columns of d, stored with the 128-byte swizzle the UMMA descriptors expect.
+fa_status map_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int d) {
+  EncodeTiledFn enc;
+  fa_status st = get_encoder(&enc);
+  if (st != FA_OK) return st;
+  const cuuint64_t gdim[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
+                              static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
+  const cuuint64_t gstride[3] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(H) * d * 2,
+                                 static_cast<cuuint64_t>(N) * H * d * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estride[4] = {1, 1, 1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gdim, gstride,
+                   box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(FA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", int(r));
+  return FA_OK;
+}
+
+// ------------------------------------------------------------ launch helpers
+std::mutex g_attr_mu;
+std::set<std::pair<const void*, int>> g_attr_done;
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device).
+template <typename Kern>
+fa_status set_smem(Kern kernel, int bytes, int dev) {
+  const void* key = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lk(g_attr_mu);
+  if (g_attr_done.count({key, dev})) return FA_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  g_attr_done.insert({key, dev});
+  return FA_OK;
+}
+
+fa_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return FA_OK;
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const fa::FwdParams& p, int dev, cudaStream_t stream) {
+  using L = fa::FwdLayout<D>;
+  auto kern = fa::fwd_kernel<D, CAUSAL>;
+  fa_status st = set_smem(kern, L::kAlloc, dev);
+  if (st != FA_OK) return st;
+  const unsigned grid = static_cast<unsigned>(p.num_qblocks) * p.B * p.H;
+  kern<<<grid, L::kThreads, L::kAlloc, stream>>>(mq, mk, mv, p);
+  return check_launch("fa_fwd kernel launch");
+}
+
+
+template <int D, bool CAUSAL>
+fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                          const CUtensorMap& mdo, const fa::BwdParams& p, int dev, cudaStream_t stream) {
+  using L = fa::BwdLayout<D>;
+  auto kern = fa::bwd_kernel<D, CAUSAL>;
+  fa_status st = set_smem(kern, L::kBytes, dev);
+  if (st != FA_OK) return st;
+  const unsigned grid = static_cast<unsigned>(p.nqt) * p.B * p.H;
+  kern<<<grid, L::kThreads, L::kBytes, stream>>>(mq, mk, mv, mdo, p);
+  return check_launch("fa_bwd main kernel launch");
+}
+
+fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                  bool causal, float scale, void* workspace, const fa::BwdWorkspace& ws, int dev,
+                  cudaStream_t stream) {
+  CUtensorMap mq, mk, mv, mdo;
+  fa_status st;
+  if ((st = map_bnhd(&mq, q, B, N, H, d)) != FA_OK) return st;
+  if ((st = map_bnhd(&mk, k, B, N, H, d)) != FA_OK) return st;
+  if ((st = map_bnhd(&mv, v, B, N, H, d)) != FA_OK) return st;
+  if ((st = map_bnhd(&mdo, dout, B, N, H, d)) != FA_OK) return st;
+  fa::BwdParams p;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.Np = (N + 127) / 128 * 128;
+  p.nqt = p.Np / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<const uint16_t*>(out);
+  p.dout = static_cast<const uint16_t*>(dout);
+  p.lse = lse;
+  char* w = static_cast<char*>(workspace);
+  p.dq_acc = reinterpret_cast<float*>(w + ws.dq_off);
+  p.lse2 = reinterpret_cast<float*>(w + ws.lse2_off);
+  p.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
+  p.dq = static_cast<uint16_t*>(dq);
+  p.dk = static_cast<uint16_t*>(dk);
+  p.dv = static_cast<uint16_t*>(dv);
+  const long long tpr = d / 8;
+  const long long pre_threads = static_cast<long long>(B) * H * p.Np * tpr;
+  const unsigned pre_blocks = static_cast<unsigned>((pre_threads + 255) / 256);
+  if (d == 64) fa::bwd_pre_kernel<64><<<pre_blocks, 256, 0, stream>>>(p);
+  else fa::bwd_pre_kernel<128><<<pre_blocks, 256, 0, stream>>>(p);
+  if ((st = check_launch("fa_bwd preprocess launch")) != FA_OK) return st;
+  if (d == 64) st = causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, p, dev, stream)
+                           : launch_bwd_main<64, false>(mq, mk, mv, mdo, p, dev, stream);
+  else st = causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, p, dev, stream)
+                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, p, dev, stream);
+  if (st != FA_OK) return st;
+  const long long cv_threads = static_cast<long long>(B) * N * H * tpr;
+  const unsigned cv_blocks = static_cast<unsigned>((cv_threads + 255) / 256);
+  if (d == 64) fa::bwd_dq_convert_kernel<64><<<cv_blocks, 256, 0, stream>>>(p);
+  else fa::bwd_dq_convert_kernel<128><<<cv_blocks, 256, 0, stream>>>(p);
+  return check_launch("fa_bwd dq convert launch");
+}
+
+int decode_splits(int B, int H, int Ncap, int sms, int* chunk_out) {
+  const long long heads = static_cast<long long>(B) * H;
+  const int min_split = (Ncap + fa::kDecodeMaxChunk - 1) / fa::kDecodeMaxChunk;
+  const int max_split = std::max(1, (Ncap + 63) / 64);  // at least 64 keys per split
+  long long ns = (static_cast<long long>(sms) * 8 + heads - 1) / std::max(1LL, heads);
+  ns = std::min<long long>(ns, max_split);
+  ns = std::max<long long>(ns, min_split);
+  ns = std::max<long long>(ns, 1);
+  int chunk = static_cast<int>((Ncap + ns - 1) / ns);
+  chunk = (chunk + 15) / 16 * 16;
+  if (chunk > fa::kDecodeMaxChunk) chunk = fa::kDecodeMaxChunk;
+  const int nsplit = (Ncap + chunk - 1) / chunk;
+  if (chunk_out) *chunk_out = chunk;
+  return nsplit;
+}
+
+size_t decode_ws_bytes(int B, int H, int d, int nsplit) {
+  if (nsplit <= 1) return 0;
+  const size_t heads = static_cast<size_t>(B) * H;
+  const size_t o_bytes = heads * nsplit * d * sizeof(float);
+  const size_t o_pad = (o_bytes + 255) / 256 * 256;
+  return o_pad + heads * nsplit * sizeof(float);
+}
+
+__global__ void timeout_probe_kernel(long long limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    fa::mbar_init(fa::smem_u32(&bar), 1);
+    fa::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // Nothing ever arrives on this barrier: the bounded wait must give up.
+    const long long t0 = clock64();
+    while (!fa::mbar_try_wait(fa::smem_u32(&bar), 0)) {
+      if (clock64() - t0 > limit) {
+        fa::report(fa::kDevTimeout, 0x7FFu, 0u);
+        break;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+// =============================================================================
+extern "C" {
+
+int fa_abi_version(void) { return kAbiVersion; }
+
+const char* fa_last_error(void) { return g_last_error.c_str(); }
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse, int B, int H,
+                 int N, int d, int causal, float scale, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "fa_fwd: negative size B=%d H=%d N=%d", B, H, N);
+  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "fa_fwd: head dim %d not supported (64 or 128)", d);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "fa_fwd: scale must be finite");
+  if (B == 0 || H == 0 || N == 0) return FA_OK;
+  if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd: null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd: q/k/v/out must be 16-byte aligned, lse 4-byte aligned");
+  const long long nqb = (static_cast<long long>(N) + 255) / 256;
+  if (nqb * B * H >= (1LL << 31) || N > (1 << 30) || H > (1 << 20))
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd: problem too large (B=%d H=%d N=%d)", B, H, N);
+  int dev = 0;
+  fa_status st = current_device(&dev, nullptr);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = map_bnhd(&mq, q, B, N, H, d)) != FA_OK) return st;
+  if ((st = map_bnhd(&mk, k, B, N, H, d)) != FA_OK) return st;
+  if ((st = map_bnhd(&mv, v, B, N, H, d)) != FA_OK) return st;
+  fa::FwdParams p;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.num_qblocks = static_cast<int>(nqb);
+  p.nkv_total = (N + 127) / 128;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return causal ? launch_fwd<64, true>(mq, mk, mv, p, dev, s) : launch_fwd<64, false>(mq, mk, mv, p, dev, s);
+  return causal ? launch_fwd<128, true>(mq, mk, mv, p, dev, s) : launch_fwd<128, false>(mq, mk, mv, p, dev, s);
+}
+
+size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
+  if (B <= 0 || H <= 0 || N <= 0 || (d != 64 && d != 128)) return 0;
+  return fa::bwd_ws_layout(B, H, N, d).total;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (B < 0 || H < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "fa_bwd: negative size B=%d H=%d N=%d", B, H, N);
+  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "fa_bwd: head dim %d not supported (64 or 128)", d);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "fa_bwd: scale must be finite");
+  if (B == 0 || H == 0 || N == 0) return FA_OK;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv)
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned4(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: tensors must be 16-byte aligned, lse 4-byte aligned");
+  const long long nkb = (static_cast<long long>(N) + 127) / 128;
+  if (nkb * B * H >= (1LL << 31) || N > (1 << 30) || H > (1 << 20))
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: problem too large (B=%d H=%d N=%d)", B, H, N);
+  const fa::BwdWorkspace ws = fa::bwd_ws_layout(B, H, N, d);
+  if (!workspace || workspace_bytes < ws.total)
+    return fail(FA_ERR_WORKSPACE, "fa_bwd: workspace needs %zu bytes, got %zu", ws.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd: workspace must be 256-byte aligned");
+  int dev = 0;
+  fa_status st = current_device(&dev, nullptr);
+  if (st != FA_OK) return st;
+  return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, N, d, causal != 0, scale, workspace, ws,
+                 dev, static_cast<cudaStream_t>(stream));
+}
+
+size_t fa_decode_workspace_size(int B, int H, int Ncap, int d) {
+  if (B <= 0 || H <= 0 || Ncap <= 0 || (d != 64 && d != 128)) return 0;
+  const int ns = decode_splits(B, H, Ncap, sm_count_or_default(), nullptr);
+  return decode_ws_bytes(B, H, d, ns);
+}
+
+fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cache_seqlens,
+                    const void* k_new, const void* v_new, void* out, float* lse, int B, int H,
+                    int Ncap, int d, int causal, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  (void)causal;  // one query at the end of the sequence sees every valid key
+  if (B < 0 || H < 0) return fail(FA_ERR_INVALID_ARG, "fa_decode: negative size B=%d H=%d", B, H);
+  if (Ncap <= 0) return fail(FA_ERR_INVALID_ARG, "fa_decode: cache capacity must be >= 1 (got %d)", Ncap);
+  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "fa_decode: head dim %d not supported (64 or 128)", d);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "fa_decode: scale must be finite");
+  if (B == 0 || H == 0) return FA_OK;
+  if (!q || !k_cache || !v_cache || !cache_seqlens || !out)
+    return fail(FA_ERR_INVALID_ARG, "fa_decode: null pointer");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    return fail(FA_ERR_INVALID_ARG, "fa_decode: k_new and v_new must both be given or both be NULL");
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (k_new && (!aligned16(k_new) || !aligned16(v_new))) || !aligned4(cache_seqlens) ||
+      (lse && !aligned4(lse)))
+    return fail(FA_ERR_INVALID_ARG, "fa_decode: bf16 tensors must be 16-byte aligned, int/float 4-byte");
+  if (H > 65535 || B > 65535) return fail(FA_ERR_INVALID_ARG, "fa_decode: B and H must be <= 65535");
+  int dev = 0, sms = 0;
+  fa_status st = current_device(&dev, &sms);
+  if (st != FA_OK) return st;
+  int chunk = 0;
+  const int ns = decode_splits(B, H, Ncap, sms, &chunk);
+  const size_t need = decode_ws_bytes(B, H, d, ns);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(FA_ERR_WORKSPACE, "fa_decode: workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FA_ERR_INVALID_ARG, "fa_decode: workspace must be 256-byte aligned");
+  fa::DecodeParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.k_cache = static_cast<uint16_t*>(k_cache);
+  p.v_cache = static_cast<uint16_t*>(v_cache);
+  p.seqlens = cache_seqlens;
+  p.k_new = static_cast<const uint16_t*>(k_new);
+  p.v_new = static_cast<const uint16_t*>(v_new);
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  p.B = B;
+  p.H = H;
+  p.Ncap = Ncap;
+  p.nsplit = ns;
+  p.chunk = chunk;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  if (ns > 1) {
+    const size_t o_bytes = static_cast<size_t>(B) * H * ns * d * sizeof(float);
+    p.part_o = static_cast<float*>(workspace);
+    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + (o_bytes + 255) / 256 * 256);
+  } else {
+    p.part_o = nullptr;
+    p.part_lse = nullptr;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const dim3 grid(ns, H, B);
+  if (d == 64) fa::decode_split_kernel<64><<<grid, 128, 0, s>>>(p);
+  else fa::decode_split_kernel<128><<<grid, 128, 0, s>>>(p);
+  if ((st = check_launch("fa_decode split kernel launch")) != FA_OK) return st;
+  if (ns > 1) {
+    const unsigned heads = static_cast<unsigned>(B) * H;
+    if (d == 64) fa::decode_merge_kernel<64><<<heads, 64, 0, s>>>(p);
+    else fa::decode_merge_kernel<128><<<heads, 128, 0, s>>>(p);
+    if ((st = check_launch("fa_decode merge kernel launch")) != FA_OK) return st;
+  }
+  return FA_OK;
+}
+
+fa_status fa_device_status(void* stream, unsigned int* site_out, unsigned int* info_out) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_device_status: stream synchronize");
+  unsigned int w[4] = {0, 0, 0, 0};
+  e = cudaMemcpyFromSymbol(w, fa::g_status, sizeof(w));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_device_status: read status word");
+  if (site_out) *site_out = w[1];
+  if (info_out) *info_out = w[2];
+  if (w[0] == 0) return FA_OK;
+  const unsigned int zero[4] = {0, 0, 0, 0};
+  e = cudaMemcpyToSymbol(fa::g_status, zero, sizeof(zero));
+  if (e != cudaSuccess) return cuda_fail(e, "fa_device_status: clear status word");
+  if (w[0] == fa::kDevTimeout)
+    return fail(FA_ERR_TIMEOUT, "device pipeline wait timed out (site 0x%x, info %u)", w[1], w[2]);
+  if (w[0] == fa::kDevBadInput)
+    return fail(FA_ERR_DEVICE_INPUT, "device input out of range (site 0x%x, batch %u)", w[1], w[2]);
+  return fail(FA_ERR_CUDA, "unknown device status %u", w[0]);
+}
+
+fa_status fa_debug_timeout_probe(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1000) limit_cycles = 1000;
+  if (limit_cycles > 4000000000LL) limit_cycles = 4000000000LL;
+  fa_status st = current_device(nullptr, nullptr);
+  if (st != FA_OK) return st;
+  timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
+  return check_launch("fa_debug_timeout_probe launch");
+}
+
+}  // extern "C"

@@ -1,0 +1,369 @@
+// Fused attention forward for sm_100a: O = softmax(scale * Q K^T, mask) V and the
+// per-row log-sum-exp, computed tile by tile with a running row max m and running
+// exp-sum l so the N x N score matrix never leaves the SM.
+//
+// Method: tiling of Q/K/V into blocks kept on chip, the blockwise softmax that
+// keeps (m, l) per row and rescales the partial output when m grows, and fusion of
+// matmul + softmax + weighted sum into one kernel ("FlashAttention优化Transformer显存
+// 与计算效率", sections 2.2.1-2.2.3); fp32 softmax accumulation with bf16 inputs
+// and outputs (same page, section 3.2); causal masking (ms-swift FA2/3 page, FA3
+// feature list). The LSE output is what the backward pass recomputes from.
+//
+// B200 design (not the pages' A100/H100 tiling):
+//  * one CTA = one (batch, head) and 256 query rows held as two 128-row tiles;
+//  * warp 8 streams K_j and V_j (128 x d bf16) through a ring of shared-memory
+//    stages with TMA (128-byte swizzle) and mbarrier full/empty pairs;
+//  * warp 9 issues tcgen05.mma from one thread: S_t = Q_t K_j^T into TMEM
+//    (fp32, 128 lanes x 128 columns per tile), then O_t += P_t V_j with P_t read
+//    straight from TMEM (bf16 packed over the first 64 columns of S_t);
+//  * warps 0-3 and 4-7 are the softmax warpgroups of tiles 0 and 1; each thread
+//    owns one query row (one TMEM lane), so row max and row sum need no shuffles.
+//    The two groups alternate with the tensor core: while one does exp, the MMA
+//    warp computes the other tile's products;
+//  * TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+d) O_1 [256+d,256+2d).
+#pragma once
+
+#include <math.h>
+
+#include "ptx.cuh"
+
+namespace fa {
+
+struct FwdParams {
+  int B, H, N;
+  int num_qblocks;   // ceil(N / 256): CTAs per (batch, head)
+  int nkv_total;     // ceil(N / 128): key tiles per head
+  float scale_log2;  // scale * log2(e)
+  uint16_t* out;     // [B, N, H, d] bf16
+  float* lse;        // [B, H, N] fp32, natural log
+};
+
+template <int D>
+struct FwdLayout {
+  static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
+  static constexpr int kStages = (D == 128) ? 4 : 6;
+  static constexpr int kQOff = 0;
+  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  // barrier indices
+  static constexpr int kQFull = 0;                      // [2]
+  static constexpr int kKVFull = 2;                     // [kStages]
+  static constexpr int kKVEmpty = 2 + kStages;          // [kStages]
+  static constexpr int kSFull = 2 + 2 * kStages;        // [2]
+  static constexpr int kPFull = kSFull + 2;             // [2]
+  static constexpr int kOFinal = kPFull + 2;            // [2]
+  static constexpr int kDrain = kOFinal + 2;            // [1]
+  static constexpr int kNumBars = kDrain + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
+  static constexpr int kThreads = 320;
+  static constexpr uint32_t kTmemCols = 512;
+};
+
+// Site ids for timeout reports.
+enum : unsigned int { kSiteFwdProducer = 0x101, kSiteFwdMma = 0x102, kSiteFwdSoftmax = 0x103 };
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(320, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using L = FwdLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_u32 = smem_u32(smem_raw);
+  const uint32_t base = (raw_u32 + 1023u) & ~1023u;
+  uint8_t* smem = smem_raw + (base - raw_u32);
+  const uint32_t sQ = base + L::kQOff;
+  const uint32_t sKV = base + L::kKVOff;
+  const uint32_t bar0 = base + L::kBarOff;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+#define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+
+  // Work unit: heaviest causal row blocks get the lowest block ids.
+  const int BH = p.B * p.H;
+  const int qb = p.num_qblocks - 1 - static_cast<int>(blockIdx.x) / BH;
+  const int bh = static_cast<int>(blockIdx.x) % BH;
+  const int b = bh / p.H;
+  const int h = bh % p.H;
+  int row0[2], nkv[2];
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    row0[t] = qb * 256 + t * 128;
+    const bool valid = row0[t] < p.N;
+    nkv[t] = !valid ? 0 : (CAUSAL ? min(row0[t] / 128 + 1, p.nkv_total) : p.nkv_total);
+  }
+  const int nkv_max = max(nkv[0], nkv[1]);
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(BAR(L::kQFull + t), 1);
+      mbar_init(BAR(L::kSFull + t), 1);
+      mbar_init(BAR(L::kPFull + t), 128);
+      mbar_init(BAR(L::kOFinal + t), 1);
+    }
+    for (int s = 0; s < L::kStages; ++s) {
+      mbar_init(BAR(L::kKVFull + s), 1);
+      mbar_init(BAR(L::kKVEmpty + s), 1);
+    }
+    mbar_init(BAR(L::kDrain), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      for (int t = 0; t < 2; ++t) {
+        if (nkv[t] == 0) continue;
+        mbar_arrive_expect_tx(BAR(L::kQFull + t), L::kTileBytes);
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_4d(sQ + t * L::kTileBytes + bx * 16384, &tmQ, BAR(L::kQFull + t), bx * 64, h,
+                      row0[t], b);
+      }
+      int it = 0;
+      for (int j = 0; j < nkv_max; ++j) {
+        bool stop = false;
+        for (int kv = 0; kv < 2; ++kv) {
+          const int s = it % L::kStages;
+          const uint32_t ph = (it / L::kStages) & 1;
+          if (!wait_bar(BAR(L::kKVEmpty + s), ph ^ 1u, abort_flag, kSiteFwdProducer)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(BAR(L::kKVFull + s), L::kTileBytes);
+          const CUtensorMap* m = kv ? &tmV : &tmK;
+          for (int bx = 0; bx < D / 64; ++bx)
+            tma_load_4d(sKV + s * L::kTileBytes + bx * 16384, m, BAR(L::kKVFull + s), bx * 64, h,
+                        j * 128, b);
+          ++it;
+        }
+        if (stop) break;
+      }
+      // Never leave the CTA with copies in flight.
+      for (int k = max(0, it - L::kStages); k < it; ++k)
+        drain_wait(BAR(L::kKVFull + k % L::kStages), (k / L::kStages) & 1);
+      for (int t = 0; t < 2; ++t)
+        if (nkv[t] > 0) drain_wait(BAR(L::kQFull + t), 0);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, 0, 0);
+      constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+      bool ok = true;
+      auto issue_qk = [&](int t, int s) {
+        const uint32_t dt = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
+          const uint64_t ad = sdesc_sw128(sQ + t * L::kTileBytes + koff, 16, 1024);
+          const uint64_t bd = sdesc_sw128(sKV + s * L::kTileBytes + koff, 16, 1024);
+          umma_ss(dt, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int s, bool acc) {
+        const uint32_t dt = tmem + 256 + t * D;
+        const uint32_t at = tmem + t * 128;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint64_t bd = sdesc_sw128(sKV + s * L::kTileBytes + kk * 2048, 16384, 1024);
+          umma_ts(dt, at + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      for (int t = 0; t < 2 && ok; ++t)
+        if (nkv[t] > 0) ok = wait_bar(BAR(L::kQFull + t), 0, abort_flag, kSiteFwdMma);
+      if (ok) {
+        // S_t for key tile 0 (ring load 0).
+        ok = wait_bar(BAR(L::kKVFull + 0), 0, abort_flag, kSiteFwdMma);
+        if (ok) {
+          tc_fence_after();
+          for (int t = 0; t < 2; ++t) {
+            if (nkv[t] == 0) continue;
+            issue_qk(t, 0);
+            umma_commit(BAR(L::kSFull + t));
+          }
+          umma_commit(BAR(L::kKVEmpty + 0));
+        }
+      }
+      for (int j = 0; j < nkv_max && ok; ++j) {
+        const int iv = 2 * j + 1, ik = 2 * j + 2;
+        const int sv = iv % L::kStages, sk = ik % L::kStages;
+        if (!wait_bar(BAR(L::kKVFull + sv), (iv / L::kStages) & 1, abort_flag, kSiteFwdMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        bool k_next = false;
+        for (int t = 0; t < 2; ++t) {
+          if (j >= nkv[t]) continue;
+          if (!wait_bar(BAR(L::kPFull + t), j & 1, abort_flag, kSiteFwdMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(t, sv, j > 0);
+          if (j + 1 < nkv[t]) {
+            if (!k_next) {
+              if (!wait_bar(BAR(L::kKVFull + sk), (ik / L::kStages) & 1, abort_flag,
+                            kSiteFwdMma)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              k_next = true;
+            }
+            issue_qk(t, sk);
+            umma_commit(BAR(L::kSFull + t));
+          } else {
+            umma_commit(BAR(L::kOFinal + t));
+          }
+        }
+        if (!ok) break;
+        umma_commit(BAR(L::kKVEmpty + sv));
+        if (k_next) umma_commit(BAR(L::kKVEmpty + sk));
+      }
+      // Let every issued MMA finish before TMEM can be released.
+      umma_commit(BAR(L::kDrain));
+      drain_wait(BAR(L::kDrain), 0);
+    }
+  } else {
+    // ------------------------------------------------------- softmax warpgroups
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;
+    const int row_g = row0[t] + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tS = tmem + t * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + t * D + lane_off;
+    const int diag_j = CAUSAL ? row0[t] / 128 : -1;
+    const float sl2 = p.scale_log2;
+    float m = -INFINITY;  // running max, log2-scaled units
+    float l = 0.f;        // running exp-sum
+    bool ok = true;
+    for (int j = 0; j < nkv[t]; ++j) {
+      ok = __all_sync(0xffffffffu,
+                      wait_bar(BAR(L::kSFull + t), j & 1, abort_flag, kSiteFwdSoftmax));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t s0[32], s1[32], s2[32], s3[32];
+      tmem_ld32(tS + 0, s0);
+      tmem_ld32(tS + 32, s1);
+      tmem_ld32(tS + 64, s2);
+      tmem_ld32(tS + 96, s3);
+      tmem_wait_ld();
+      reg_fence32(s0);
+      reg_fence32(s1);
+      reg_fence32(s2);
+      reg_fence32(s3);
+      float x[128];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        x[c] = __uint_as_float(s0[c]) * sl2;
+        x[32 + c] = __uint_as_float(s1[c]) * sl2;
+        x[64 + c] = __uint_as_float(s2[c]) * sl2;
+        x[96 + c] = __uint_as_float(s3[c]) * sl2;
+      }
+      const int kbase = j * 128;
+      if (j == diag_j || kbase + 128 > p.N) {
+        const int lim = CAUSAL ? min(row_g, p.N - 1) : p.N - 1;
+#pragma unroll
+        for (int c = 0; c < 128; ++c)
+          if (kbase + c > lim) x[c] = -INFINITY;
+      }
+      float mx = x[0];
+#pragma unroll
+      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+      const float m_new = fmaxf(m, mx);
+      const float ms = (m_new == -INFINITY) ? 0.f : m_new;
+      const float alpha = ex2_approx(m - ms);
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        x[c] = ex2_approx(x[c] - ms);
+        rs += x[c];
+      }
+      if (j > 0 && __any_sync(0xffffffffu, m_new > m)) {
+        // The running max grew: rescale this row's partial output in TMEM.
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          tmem_st32(tO + cc * 32, o);
+        }
+      }
+      l = l * alpha + rs;
+      m = m_new;
+      uint32_t pk0[32], pk1[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        pk0[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
+        pk1[c] = pack_bf16x2(x[64 + 2 * c], x[64 + 2 * c + 1]);
+      }
+      tmem_st32(tS + 0, pk0);
+      tmem_st32(tS + 32, pk1);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(BAR(L::kPFull + t));
+    }
+    if (ok && nkv[t] > 0) {
+      ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kOFinal + t), 0, abort_flag, kSiteFwdSoftmax));
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+        const bool row_ok = row_g < p.N;
+        uint16_t* orow = p.out + ((static_cast<size_t>(b) * p.N + row_g) * p.H + h) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l,
+                                __uint_as_float(o[2 * c + 1]) * inv_l);
+          if (row_ok) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4)
+              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          }
+        }
+        if (row_ok) {
+          const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
+          p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + row_g] = lse;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+#undef BAR
+}
+
+}  // namespace fa

@@ -1,0 +1,229 @@
+"""Python binding of libfa.so: argument marshalling only.
+
+Every function here checks torch tensor metadata (device, dtype, contiguity,
+shapes), allocates outputs and workspaces with torch (device memory is the only
+thing PyTorch provides), and calls the C ABI declared in include/fa.h on the
+current CUDA stream. All arithmetic runs in the library's CUDA kernels; there is
+no CPU or PyTorch fallback: a missing library or an unsupported device raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["FAError", "load_library", "fwd", "bwd", "decode", "bwd_workspace_size",
+           "decode_workspace_size", "device_status", "debug_timeout_probe", "LIB_PATH",
+           "declared_symbols"]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
+
+FA_OK = 0
+STATUS_NAMES = {0: "FA_OK", 1: "FA_ERR_INVALID_ARG", 2: "FA_ERR_UNSUPPORTED", 3: "FA_ERR_CUDA",
+                4: "FA_ERR_WORKSPACE", 5: "FA_ERR_TIMEOUT", 6: "FA_ERR_DEVICE_INPUT"}
+
+_c_void_p = ctypes.c_void_p
+_c_int = ctypes.c_int
+_c_float = ctypes.c_float
+_c_size_t = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/fa.h
+_SIGNATURES = {
+    "fa_fwd": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                        _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p]),
+    "fa_bwd_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
+    "fa_bwd": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                        _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                        _c_float, _c_void_p, _c_size_t, _c_void_p]),
+    "fa_decode_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
+    "fa_decode": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                           _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                           _c_float, _c_void_p, _c_size_t, _c_void_p]),
+    "fa_last_error": (ctypes.c_char_p, []),
+    "fa_device_status": (_c_int, [_c_void_p, ctypes.POINTER(ctypes.c_uint),
+                                  ctypes.POINTER(ctypes.c_uint)]),
+    "fa_debug_timeout_probe": (_c_int, [ctypes.c_longlong, _c_void_p]),
+    "fa_abi_version": (_c_int, []),
+}
+
+
+def declared_symbols():
+    """Names of the C entry points this binding expects (those of include/fa.h)."""
+    return sorted(_SIGNATURES)
+
+
+class FAError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        self.status = status
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH):
+    """Load libfa.so (once) and attach the C signatures. Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"CUDA library not built: {path} is missing. Build it with "
+            "`python -m exact_attention_155_b200.build` (or __graft_entry__.build()).")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != FA_OK:
+        msg = load_library().fa_last_error()
+        raise FAError(status, msg.decode() if msg else "")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _require(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype} (got {t.dtype}); inputs and outputs share one dtype")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _scale(scale, d):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
+        scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+        lse: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Exact attention forward. q, k, v: [B, N, H, d] bf16 CUDA tensors.
+
+    Returns (out [B, N, H, d] bf16, lse [B, H, N] fp32). scale=None -> 1/sqrt(d).
+    """
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require(t, name)
+    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
+        raise ValueError(f"q, k, v must all be [B, N, H, d] with equal shapes "
+                         f"(got {tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)})")
+    B, N, H, d = q.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    _require(out, "out")
+    _require(lse, "lse", torch.float32)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
+                          int(bool(causal)), _scale(scale, d), _stream(stream)))
+    return out, lse
+
+
+def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().fa_bwd_workspace_size(B, H, N, d))
+
+
+def bwd(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = None,
+        dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Attention backward by recomputation. Returns (dq, dk, dv), bf16 [B, N, H, d]."""
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _require(t, name)
+        if t.shape != q.shape:
+            raise ValueError(f"{name} must have q's shape {tuple(q.shape)}")
+    _require(lse, "lse", torch.float32)
+    B, N, H, d = q.shape
+    if tuple(lse.shape) != (B, H, N):
+        raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
+        _require(t, name)
+    lib = load_library()
+    need = int(lib.fa_bwd_workspace_size(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                          _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
+                          _scale(scale, d), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def decode_workspace_size(B: int, H: int, Ncap: int, d: int) -> int:
+    return int(load_library().fa_decode_workspace_size(B, H, Ncap, d))
+
+
+def decode(q, k_cache, v_cache, cache_seqlens, k_new=None, v_new=None, causal: bool = True,
+           scale: Optional[float] = None, out=None, lse=None, workspace=None, stream=None):
+    """One KV-cache decode step (flash_attn_with_kvcache semantics).
+
+    q: [B, 1, H, d]; k_cache, v_cache: [B, Ncap, H, d]; cache_seqlens: int32 [B] on the
+    device (valid rows before the append). With k_new / v_new ([B, 1, H, d]) the row is
+    appended at cache_seqlens[b]. Returns (out [B, 1, H, d] bf16, lse [B, H] fp32).
+    """
+    _require(q, "q")
+    _require(k_cache, "k_cache")
+    _require(v_cache, "v_cache")
+    _require(cache_seqlens, "cache_seqlens", torch.int32)
+    B, one, H, d = q.shape
+    if one != 1 or k_cache.dim() != 4 or k_cache.shape != v_cache.shape \
+            or k_cache.shape[0] != B or k_cache.shape[2] != H or k_cache.shape[3] != d:
+        raise ValueError("q must be [B,1,H,d] and caches [B,Ncap,H,d]")
+    if tuple(cache_seqlens.shape) != (B,):
+        raise ValueError("cache_seqlens must be int32 [B]")
+    Ncap = k_cache.shape[1]
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new must be given together")
+    if k_new is not None:
+        _require(k_new, "k_new")
+        _require(v_new, "v_new")
+        if k_new.shape != q.shape or v_new.shape != q.shape:
+            raise ValueError("k_new and v_new must be [B, 1, H, d]")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    _require(out, "out")
+    _require(lse, "lse", torch.float32)
+    lib = load_library()
+    need = int(lib.fa_decode_workspace_size(B, H, Ncap, d))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    with torch.cuda.device(q.device):
+        _check(lib.fa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens),
+                             _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(lse), B, H, Ncap, d,
+                             int(bool(causal)), _scale(scale, d), _ptr(workspace), ws_bytes,
+                             _stream(stream)))
+    return out, lse
+
+
+def device_status(stream=None):
+    """Synchronise the stream and return (status, site, info) from the device status word."""
+    lib = load_library()
+    site, info = ctypes.c_uint(0), ctypes.c_uint(0)
+    st = lib.fa_device_status(_stream(stream), ctypes.byref(site), ctypes.byref(info))
+    return st, site.value, info.value
+
+
+def debug_timeout_probe(limit_cycles: int, stream=None):
+    """Launch the diagnostic kernel whose wait must time out (see include/fa.h)."""
+    _check(load_library().fa_debug_timeout_probe(int(limit_cycles), _stream(stream)))

@@ -1,0 +1,144 @@
+/*
+ * fa.h - C ABI of the B200 (sm_100a) exact-attention library (libfa.so).
+ *
+ * The library computes exact scaled-dot-product attention,
+ *     O = softmax(scale * Q K^T [+ causal mask]) V,
+ * the definition printed on every page it follows (e.g. the opening formula of
+ * "Flash-Attention 2/3在ms-swift中的集成与性能提升" and section 一 of the Qwen
+ * flash_attn explainer), computed tile by tile with a running row max and row sum
+ * ("FlashAttention优化Transformer显存与计算效率", sections 2.2.1-2.2.3) so the N x N
+ * score matrix never reaches global memory.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Tensors are DEVICE pointers to contiguous row-major arrays. Q, K, V, O and their
+ *    gradients are bf16 (passed as void*, 2 bytes per element) in the layout
+ *    [B, N, H, d] = (batch, seq_len, heads, head_dim), the layout of section 1.1 of
+ *    "ms-swift长文本训练优化，Flash-Attention显存省一半". Every bf16 pointer must be
+ *    16-byte aligned; float pointers 4-byte aligned.
+ *  - d (head_dim) must be 64 or 128. The device must be compute capability 10.0
+ *    (B200, sm_100a).
+ *  - scale is the softmax scale; any finite value. (The pages' softmax_scale=None
+ *    default, 1/sqrt(d), is applied by the Python binding, not here.)
+ *  - LSE is the natural-log log-sum-exp of each query row's scaled scores over its
+ *    visible keys, fp32, laid out [B, H, N]. A row with no visible key gets -inf.
+ *  - causal != 0 masks key j for query i when j > i (for decode, the single new
+ *    query sees every valid key, so causal changes nothing there).
+ *  - stream is a cudaStream_t (NULL = legacy default stream). Every call only
+ *    enqueues work on that stream and returns without synchronising.
+ *  - Ownership: the caller allocates and owns every buffer, including workspaces;
+ *    the library allocates no device memory and keeps no per-call state. Inputs are
+ *    read-only except the KV cache rows that fa_decode appends.
+ *  - Errors: argument problems are detected on the host before anything is
+ *    launched and return a non-zero status with a message from fa_last_error().
+ *    Problems only visible on the device (a cache_seqlens value out of range, an
+ *    internal pipeline wait that timed out) are recorded in a device status word
+ *    and read back by fa_device_status().
+ *  - Empty problems (B, N or H equal to 0) return FA_OK without launching.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,   /* null pointer, bad size, misalignment, non-finite scale */
+  FA_ERR_UNSUPPORTED = 2,   /* d not in {64,128}, or device is not sm_100 */
+  FA_ERR_CUDA = 3,          /* a CUDA runtime/driver call or kernel launch failed */
+  FA_ERR_WORKSPACE = 4,     /* workspace pointer null or smaller than required */
+  FA_ERR_TIMEOUT = 5,       /* (device) a pipeline wait gave up; results are invalid */
+  FA_ERR_DEVICE_INPUT = 6   /* (device) cache_seqlens out of range / cache full */
+} fa_status;
+
+/*
+ * Fused forward: out = softmax(scale*Q K^T, mask) V and lse, in one kernel.
+ *   q, k, v : [B, N, H, d] bf16 (read)        out : [B, N, H, d] bf16 (written)
+ *   lse     : [B, H, N] fp32 (written)
+ * Follows the forward pass of the pages: tiling + blockwise softmax + fusion
+ * ("FlashAttention优化Transformer显存与计算效率" 2.2), fp32 softmax accumulation with
+ * bf16 in/out (same page 3.2), causal flag (flash_attn_func(..., causal=True)).
+ */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                 int B, int H, int N, int d, int causal, float scale, void* stream);
+
+/* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator and
+ * the per-row D = rowsum(dO * O) vector). Pure function of its arguments. */
+size_t fa_bwd_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward with recomputation: from q, k, v, out, dout and the forward's lse,
+ * rebuild P = exp(scale*Q K^T - lse) tile by tile (the score matrix is recomputed,
+ * not stored, as the pages' "重计算 / Recomputation" item describes) and write
+ *   dv = P^T dO,  dk = scale * dS^T Q,  dq = scale * dS K,
+ *   where dS = P * (dO V^T - D),  D_i = sum_c dO_ic O_ic.
+ *   q, k, v, out, dout : [B, N, H, d] bf16 (read);  lse : [B, H, N] fp32 (read)
+ *   dq, dk, dv         : [B, N, H, d] bf16 (written)
+ *   workspace          : >= fa_bwd_workspace_size(B,H,N,d) bytes, 256-byte aligned;
+ *                        contents on entry are ignored and left undefined.
+ * The dq accumulation order across key tiles is not fixed (fp32 atomics), so dq
+ * may differ in the last bits between runs; dk and dv are bitwise repeatable.
+ */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of device workspace fa_decode needs (split partials); may be 0. Depends on
+ * the current device's SM count, so query it on the device that will run. */
+size_t fa_decode_workspace_size(int B, int H, int Ncap, int d);
+
+/*
+ * One KV-cache decode step (flash_attn_with_kvcache, section 推理优化与KV缓存 of
+ * "FlashAttention与MindSpore 2.0全场景融合方案"):
+ *   q                : [B, 1, H, d] bf16 (read)
+ *   k_cache, v_cache : [B, Ncap, H, d] bf16; rows >= the valid length are ignored
+ *   cache_seqlens    : [B] int32 DEVICE array, valid rows before this step
+ *   k_new, v_new     : [B, 1, H, d] bf16 or both NULL. When given, they are written
+ *                      into the caches at row cache_seqlens[b] and the query attends
+ *                      cache_seqlens[b] + 1 rows; otherwise cache_seqlens[b] rows.
+ *                      cache_seqlens itself is not modified.
+ *   out              : [B, 1, H, d] bf16 (written); lse : [B, H] fp32 or NULL
+ *   workspace        : >= fa_decode_workspace_size(B,H,Ncap,d) bytes (may be NULL
+ *                      when that size is 0), 256-byte aligned.
+ * A batch entry with no valid row gets out = 0 and lse = -inf. A cache_seqlens
+ * value < 0 or > Ncap, or == Ncap with k_new given, is recorded as
+ * FA_ERR_DEVICE_INPUT in the device status word; that entry then attends nothing
+ * and appends nothing.
+ */
+fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cache_seqlens,
+                    const void* k_new, const void* v_new, void* out, float* lse, int B, int H,
+                    int Ncap, int d, int causal, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* Message for the last non-OK status returned on the calling host thread. */
+const char* fa_last_error(void);
+
+/*
+ * Synchronises `stream`, then reads and clears the device status word of the
+ * current device. Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_DEVICE_INPUT or FA_ERR_CUDA.
+ * If site_out / info_out are non-NULL they receive the reporting site id and an
+ * extra value (the CTA or batch index).
+ */
+fa_status fa_device_status(void* stream, unsigned int* site_out, unsigned int* info_out);
+
+/*
+ * Diagnostic: launches one CTA that waits on a barrier nothing will ever complete,
+ * with its wait limit set to about `limit_cycles` clock cycles (clamped to
+ * [1e3, 4e9]). The kernel gives up, records FA_ERR_TIMEOUT in the device status
+ * word and exits; it exists so tests can check the timeout path without hanging
+ * or faulting a GPU.
+ */
+fa_status fa_debug_timeout_probe(long long limit_cycles, void* stream);
+
+/* Library ABI version (incremented on any signature change). */
+int fa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */

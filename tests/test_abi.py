@@ -1,0 +1,132 @@
+"""C ABI checks that need no GPU: the library builds, loads and exports every entry
+point include/fa.h declares; host-side argument validation returns the documented
+status before anything touches a device."""
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from exact_attention_155_b200 import build as fa_build
+from exact_attention_155_b200 import ops
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "fa.h")
+
+FA_OK, INVALID, UNSUPPORTED, CUDA, WORKSPACE = 0, 1, 2, 3, 4
+P16 = ctypes.c_void_p(0x10000)   # fake, 16-byte aligned: never dereferenced on the host
+P_ODD = ctypes.c_void_p(0x10008)  # 8-byte aligned only
+NULL = None
+S0 = ctypes.c_void_p(0)
+
+
+def _header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z_0-9]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    fa_build.build()
+    return ops.load_library()
+
+
+def test_header_and_binding_agree():
+    assert _header_functions() == ops.declared_symbols()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _header_functions():
+        assert hasattr(lib, name), name
+    assert lib.fa_abi_version() == 1
+
+
+def test_bwd_workspace_size_is_pure_and_padded(lib):
+    # dQ accumulator [B,H,Np,d] fp32 + two [B,H,Np] fp32 vectors, Np = roundup(N, 128).
+    for (B, H, N, d) in [(1, 2, 128, 64), (2, 3, 129, 128), (1, 32, 16384, 128)]:
+        Np = (N + 127) // 128 * 128
+        rows = B * H * Np
+        r256 = lambda x: (x + 255) // 256 * 256
+        expect = r256(rows * d * 4) + 2 * r256(rows * 4)
+        assert lib.fa_bwd_workspace_size(B, H, N, d) == expect
+    assert lib.fa_bwd_workspace_size(1, 1, 128, 96) == 0
+    assert lib.fa_bwd_workspace_size(0, 1, 128, 64) == 0
+
+
+def _fwd(lib, q=P16, k=P16, v=P16, o=P16, lse=P16, B=1, H=1, N=128, d=64, causal=0, scale=0.125):
+    return lib.fa_fwd(q, k, v, o, lse, B, H, N, d, causal, scale, S0)
+
+
+def test_fwd_argument_errors(lib):
+    assert _fwd(lib, d=96) == UNSUPPORTED
+    assert b"head dim" in lib.fa_last_error()
+    assert _fwd(lib, N=-1) == INVALID
+    assert _fwd(lib, scale=math.inf) == INVALID
+    assert _fwd(lib, scale=math.nan) == INVALID
+    assert _fwd(lib, q=NULL) == INVALID
+    assert _fwd(lib, o=P_ODD) == INVALID
+    assert b"aligned" in lib.fa_last_error()
+    # Empty problems are a no-op, even with null pointers.
+    assert _fwd(lib, q=NULL, k=NULL, v=NULL, o=NULL, lse=NULL, N=0) == FA_OK
+    assert _fwd(lib, B=0) == FA_OK
+
+
+def _bwd(lib, ws=P16, ws_bytes=1 << 40, d=64, N=128, dq=P16, scale=0.125):
+    return lib.fa_bwd(P16, P16, P16, P16, P16, P16, dq, P16, P16, 1, 2, N, d, 0, scale, ws,
+                      ws_bytes, S0)
+
+
+def test_bwd_argument_errors(lib):
+    assert _bwd(lib, d=32) == UNSUPPORTED
+    assert _bwd(lib, dq=NULL) == INVALID
+    assert _bwd(lib, dq=P_ODD) == INVALID
+    assert _bwd(lib, ws=NULL) == WORKSPACE
+    need = lib.fa_bwd_workspace_size(1, 2, 128, 64)
+    assert _bwd(lib, ws_bytes=need - 1) == WORKSPACE
+    assert b"workspace" in lib.fa_last_error()
+    assert _bwd(lib, ws=ctypes.c_void_p(0x10010)) == INVALID  # not 256-byte aligned
+    assert _bwd(lib, scale=math.inf) == INVALID
+
+
+def _dec(lib, q=P16, kn=NULL, vn=NULL, seq=P16, Ncap=2048, d=64, B=2):
+    return lib.fa_decode(q, P16, P16, seq, kn, vn, P16, NULL, B, 16, Ncap, d, 1, 0.125, NULL, 0, S0)
+
+
+def test_decode_argument_errors(lib):
+    assert _dec(lib, d=80) == UNSUPPORTED
+    assert _dec(lib, Ncap=0) == INVALID
+    assert _dec(lib, kn=P16, vn=NULL) == INVALID
+    assert b"both" in lib.fa_last_error()
+    assert _dec(lib, q=P_ODD) == INVALID
+    assert _dec(lib, seq=NULL) == INVALID
+    assert _dec(lib, B=0) == FA_OK
+
+
+def test_decode_workspace_size_without_device(lib):
+    # No GPU here: the split choice uses 148 SMs. A full-length sweep (B=32, H=16,
+    # 2048 rows) splits each head in 3; tiny problems need no workspace.
+    ws = lib.fa_decode_workspace_size(32, 16, 2048, 64)
+    assert ws > 0
+    heads, ns, d = 32 * 16, 3, 64
+    assert ws == (heads * ns * d * 4 + 255) // 256 * 256 + heads * ns * 4
+    assert lib.fa_decode_workspace_size(1, 1, 16, 64) == 0
+
+
+def test_calls_without_a_gpu_report_an_error_not_a_crash(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = _fwd(lib)
+    assert st in (CUDA, UNSUPPORTED)
+    assert lib.fa_last_error()
+
+
+def test_binding_raises_when_library_missing(tmp_path):
+    saved = ops._lib
+    ops._lib = None
+    try:
+        with pytest.raises(RuntimeError, match="not built"):
+            ops.load_library(str(tmp_path / "missing.so"))
+    finally:
+        ops._lib = saved
