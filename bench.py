@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path on B200.
+
+One step = the long-context causal training step: fused forward (O and LSE) plus
+the recompute backward (dQ, dK, dV) at B=1, H=32, N=16384, d=128, bf16, on
+synthetic N(0,1) inputs already resident in HBM. The metric is attention TFLOP/s
+with the algorithmic count 4*B*H*N^2*d/2 for the causal forward and 2.5x that for
+the backward. The same JSON line also reports, measured in the same run:
+  * "roofline": the backward main kernel (the step's dominant kernel) timed with
+    CUDA events on its launch stream inside the timed region;
+  * "e2e": the step through the public API from pinned host buffers, with the
+    host->device copies of q, k, v, dout and the device->host copies of out, lse,
+    dq, dk, dv inside the timed region;
+  * "parts": the causal prefill forward (B=1, H=32, N=8192, d=128) and the
+    KV-cache decode sweep (B=32, H=16, d=64, 2048 cached rows) with their own
+    rooflines, and the per-step latency of the 100-step incremental decode;
+  * "cpu_baseline": the float64 CPU oracle on a bounded sample of the same step.
+
+Multi-GPU: every rank runs an independent replica (the path has no exchange
+step); value is the sum over ranks divided by the slowest rank's time.
+
+--impl reference times the float64 oracle itself (the only reference this
+method has) on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOP/s fwd/bwd (causal, bf16) and decode GB/s; % of B200 roofline"
+WORKLOAD = dict(name="train", B=1, H=32, N=16384, d=128, causal=True)
+PREFILL = dict(B=1, H=32, N=8192, d=128, causal=True)
+SWEEP = dict(B=32, H=16, d=64, Ncap=2048, seqlen=2048)
+STEPS5 = dict(B=2, H=16, d=64, Ncap=2048, steps=100)
+
+# DRAM bytes per launch of the backward main kernel from an ncu capture, valid only
+# for the kernel source it was taken on (sha256 of csrc/bwd.cuh).
+BWD_TRAFFIC = {"src_sha256": None, "bytes_per_launch": None, "profile": None}
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def fwd_flops(B, H, N, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), tf_burst=float(p["bf16_tflops"]),
+                    tf_sustained=float(p["bf16_tflops_sustained"]), source="measured")
+    except Exception:
+        return dict(hbm=6650.0, tf_burst=1590.0, tf_sustained=1400.0, source="fallback")
+
+
+def src_sha(rel):
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+# ----------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clock, power and throttle reasons (200 ms period)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index):
+        self.proc = None
+        self.lines = []
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            sel = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            sel = str(device_index)
+        self.cmd = ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
+                    "--format=csv,noheader,nounits", "-lms", "200"]
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except Exception:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.strip().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(parts[1]), smax=float(parts[2]), power=float(parts[3]),
+                                 flags=parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        # Samples under load: power well above idle; fall back to all samples.
+        pmax = max(r["power"] for r in rows)
+        load = [r for r in rows if r["power"] >= 0.5 * pmax] or rows
+        reasons = sorted({self.NAMES[i] for r in load for i, f in enumerate(r["flags"])
+                          if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["smax"] for r in rows), "reasons": reasons,
+                "samples": len(load), "power_w_max": pmax}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def oracle_sample(target_s=6.0, max_n=None):
+    """Time the float64 oracle on one head of the causal training step, restricted to
+    a causal prefix of Ns rows (an independent sub-problem of the same workload).
+    Ns grows until one forward+backward takes about target_s seconds."""
+    import numpy as np
+    import oracle
+    from exact_attention_155_b200.inputs import attention_inputs, to_f64
+    w = WORKLOAD
+    d = w["d"]
+    scale = 1.0 / math.sqrt(d)
+    inp = attention_inputs(1, w["N"], 1, d, seed=1004)
+    full = {n: to_f64(inp[n]) for n in ("q", "k", "v", "dout")}
+    ns = 1024
+    limit = max_n or w["N"]
+    while True:
+        sub = {n: full[n][:, :ns] for n in full}
+        t0 = time.perf_counter()
+        oracle.attention_forward(sub["q"], sub["k"], sub["v"], causal=True, scale=scale)
+        oracle.attention_backward(sub["q"], sub["k"], sub["v"], sub["dout"], causal=True, scale=scale)
+        dt = time.perf_counter() - t0
+        if dt * 4 > target_s or ns * 2 > limit:
+            break
+        ns *= 2
+    flops = 3.5 * fwd_flops(1, 1, ns, d, True)
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        cores = os.cpu_count() or 1
+
+    def run_once():
+        sub = {n: full[n][:, :ns] for n in full}
+        t0 = time.perf_counter()
+        oracle.attention_forward(sub["q"], sub["k"], sub["v"], causal=True, scale=scale)
+        oracle.attention_backward(sub["q"], sub["k"], sub["v"], sub["dout"], causal=True, scale=scale)
+        return time.perf_counter() - t0
+
+    sample = (f"float64 oracle fwd+bwd of 1 of {w['B'] * w['H']} heads, causal prefix of "
+              f"{ns} of {w['N']} rows (d={d})")
+    return run_once, flops, int(cores), sample, dt
+
+
+def run_reference(args, rank):
+    if rank != 0:
+        return
+    run_once, flops, cores, sample, _ = oracle_sample(target_s=4.0)
+    for _ in range(max(0, args.warmup)):
+        run_once()
+    times = [run_once() for _ in range(max(1, args.steps))]
+    mean = statistics.mean(times)
+    value = flops / mean / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": mean * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(args.gpus),
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(n):
+    w = WORKLOAD
+    return {"workload": (f"causal training step (fwd+bwd): B={w['B']} H={w['H']} N={w['N']} "
+                         f"d={w['d']} bf16"),
+            "B": w["B"], "H": w["H"], "N": w["N"], "d": w["d"], "causal": True,
+            "global_batch": w["B"] * n, "seq_len": w["N"],
+            "l2": "inputs larger than L2 (q, k, v, dout: 4 x 128 MiB per step)",
+            "parallelism": f"replicas x{n}"}
+
+
+# ----------------------------------------------------------------- GPU timing
+def timed_events(torch, fn, reps, flush=None):
+    """Median device time (ms) of fn over reps, CUDA events on the current stream."""
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    return statistics.median(times)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    import exact_attention_155_b200 as fa
+    from exact_attention_155_b200.inputs import attention_inputs, decode_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+    w = WORKLOAD
+    B, H, N, d = w["B"], w["H"], w["N"], w["d"]
+    scale = 1.0 / math.sqrt(d)
+    f_fwd = fwd_flops(B, H, N, d, True)
+    f_bwd = 2.5 * f_fwd
+    f_step = f_fwd + f_bwd
+
+    inp = attention_inputs(B, N, H, d, seed=1004 + rank)
+    host = {n: inp[n].pin_memory() for n in ("q", "k", "v", "dout")}
+    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "dout"))
+    out = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(fa.bwd_workspace_size(B, H, N, d), dtype=torch.uint8, device=dev)
+
+    def step(ev=None):
+        if ev is None:
+            fa.fwd(q, k, v, causal=True, scale=scale, out=out, lse=lse)
+            fa.bwd(q, k, v, out, do, lse, causal=True, scale=scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+        else:
+            ev[0].record()
+            fa.fwd(q, k, v, causal=True, scale=scale, out=out, lse=lse)
+            ev[1].record()
+            fa.bwd(q, k, v, out, do, lse, causal=True, scale=scale, dq=dq, dk=dk, dv=dv,
+                   workspace=ws, main_events=(ev[2], ev[3]))
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    sampler = ClockSampler(local_rank)
+    barrier()
+    sampler.start()
+    torch.cuda.synchronize()
+    barrier()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record()
+    for i in range(K):
+        step(evs[i])
+    t_stop.record()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    elapsed_ms = max_over_ranks(t_start.elapsed_time(t_stop))
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    ms_per_step = elapsed_ms / K
+    value = world * f_step * K / (elapsed_ms * 1e-3) / 1e12
+    status = fa.device_status()[0]
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    achieved = f_bwd / (bwd_main_ms * 1e-3) / 1e12
+    traffic = None
+    if BWD_TRAFFIC["src_sha256"] == src_sha("exact_attention_155_b200/csrc/bwd.cuh"):
+        traffic = BWD_TRAFFIC["bytes_per_launch"]
+    roofline = {"kernel": "bwd_kernel<128,causal>", "bound": "tensor", "achieved": achieved,
+                "peak": peaks["tf_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["tf_sustained"],
+                "peak_kind": f"bf16 dense, sustained, of {peaks['source']}",
+                "traffic": traffic, "avg_launch_ms": bwd_main_ms,
+                "algorithmic_flop_per_launch": f_bwd}
+
+    # ---- end to end through the public API from pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        hout = torch.empty_like(out, device="cpu").pin_memory()
+        hlse = torch.empty_like(lse, device="cpu").pin_memory()
+        hdq, hdk, hdv = (torch.empty_like(x, device="cpu").pin_memory() for x in (dq, dk, dv))
+
+        def e2e_step():
+            for n, dst in (("q", q), ("k", k), ("v", v), ("dout", do)):
+                dst.copy_(host[n], non_blocking=True)
+            fa.fwd(q, k, v, causal=True, scale=scale, out=out, lse=lse)
+            fa.bwd(q, k, v, out, do, lse, causal=True, scale=scale, dq=dq, dk=dk, dv=dv, workspace=ws)
+            for src, dst in ((out, hout), (lse, hlse), (dq, hdq), (dk, hdk), (dv, hdv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        Ke = max(3, K // 4)
+        barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(Ke):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
+        e2e_ms = max_over_ranks(a.elapsed_time(b))
+        h2d = sum(host[n].numel() * host[n].element_size() for n in host)
+        d2h = sum(x.numel() * x.element_size() for x in (out, lse, dq, dk, dv))
+        e2e = {"value": world * f_step * Ke / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": e2e_ms / Ke, "steps": Ke}
+        del hout, hlse, hdq, hdk, hdv
+
+    # ---- parts: prefill forward, decode sweep, incremental decode steps
+    parts = None
+    if not args.no_parts:
+        del dq, dk, dv, ws
+        p = PREFILL
+        pin = attention_inputs(p["B"], p["N"], p["H"], p["d"], seed=1003)
+        pq, pk, pv = (pin[n].to(dev) for n in ("q", "k", "v"))
+        pout, plse = torch.empty_like(pq), torch.empty((p["B"], p["H"], p["N"]), device=dev)
+        for _ in range(3):
+            fa.fwd(pq, pk, pv, causal=True, scale=scale, out=pout, lse=plse)
+        pms = timed_events(torch, lambda: fa.fwd(pq, pk, pv, causal=True, scale=scale, out=pout,
+                                                 lse=plse), 20)
+        ptf = fwd_flops(p["B"], p["H"], p["N"], p["d"], True) / (pms * 1e-3) / 1e12
+        del pq, pk, pv, pout, plse
+        s = SWEEP
+        kc, vc, qs, _, _ = decode_inputs(s["B"], s["H"], s["d"], s["Ncap"], 1, seed=1005)
+        kc, vc, qd = kc.to(dev), vc.to(dev), qs[0].to(dev)
+        seq = torch.full((s["B"],), s["seqlen"], dtype=torch.int32, device=dev)
+        dws = torch.empty(max(1, fa.decode_workspace_size(s["B"], s["H"], s["Ncap"], s["d"])),
+                          dtype=torch.uint8, device=dev)
+        dout_ = torch.empty_like(qd)
+        dlse = torch.empty((s["B"], s["H"]), device=dev)
+        flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        dec = lambda: fa.decode(qd, kc, vc, seq, scale=1 / 8, out=dout_, lse=dlse, workspace=dws)
+        for _ in range(3):
+            dec()
+        dms = timed_events(torch, dec, 30, flush=flush)
+        dbytes = 2 * s["B"] * s["H"] * s["seqlen"] * s["d"] * 2
+        dgbs = dbytes / (dms * 1e-3) / 1e9
+        del kc, vc, flush
+        c5 = STEPS5
+        kc, vc, qs, ks, vs = decode_inputs(c5["B"], c5["H"], c5["d"], c5["Ncap"], c5["steps"], seed=1005)
+        kc, vc, qs, ks, vs = kc.to(dev), vc.to(dev), qs.to(dev), ks.to(dev), vs.to(dev)
+        seqs = [torch.full((c5["B"],), t, dtype=torch.int32, device=dev) for t in range(c5["steps"])]
+        o5 = torch.empty_like(qs[0])
+        l5 = torch.empty((c5["B"], c5["H"]), device=dev)
+        ws5 = torch.empty(max(1, fa.decode_workspace_size(c5["B"], c5["H"], c5["Ncap"], c5["d"])),
+                          dtype=torch.uint8, device=dev)
+
+        def steps100():
+            for t in range(c5["steps"]):
+                fa.decode(qs[t], kc, vc, seqs[t], ks[t], vs[t], scale=1 / 8, out=o5, lse=l5,
+                          workspace=ws5)
+        steps100()
+        sms = timed_events(torch, steps100, 5)
+        parts = {
+            "prefill_fwd": {"workload": "causal fwd B=1 H=32 N=8192 d=128", "value": ptf,
+                            "unit": "TFLOP/s", "ms": pms, "roofline_bound": "tensor",
+                            "frac": ptf / peaks["tf_burst"],
+                            "peak": peaks["tf_burst"],
+                            "peak_kind": f"bf16 dense, burst, of {peaks['source']}"},
+            "train_fwd_in_step": {"value": f_fwd / (fwd_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                                  "ms": fwd_ms},
+            "decode_sweep": {"workload": "decode B=32 H=16 d=64, 2048 cached rows, no append",
+                             "value": dgbs, "unit": "GB/s", "us": dms * 1e3,
+                             "roofline_bound": "hbm", "frac": dgbs / peaks["hbm"],
+                             "peak": peaks["hbm"], "peak_kind": f"HBM copy, of {peaks['source']}",
+                             "l2": "flushed (512 MiB write) before every call"},
+            "decode_steps": {"workload": "decode B=2 H=16 d=64 cap 2048, 100 appending steps",
+                             "us_per_step": sms * 1e3 / c5["steps"],
+                             "gb_s": 8192 * sum(t + 1 for t in range(c5["steps"]))
+                             / (sms * 1e-3) / 1e9},
+        }
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        run_once, flops, cores, sample, _ = oracle_sample(target_s=12.0)
+        dt = min(run_once() for _ in range(1))
+        cpu = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+               "sample": sample, "seconds": dt}
+
+    launches_per_step = 4  # fwd kernel + bwd preprocess, main and dq-convert kernels
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(world), "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+        "gpu_launches": launches_per_step * K, "clocks": clocks, "parts": parts,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-parts", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warmup raised to 3 (minimum)")
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

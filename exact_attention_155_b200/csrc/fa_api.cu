@@ -185,7 +185,7 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
 fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                   const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                   bool causal, float scale, void* workspace, const fa::BwdWorkspace& ws, int dev,
-                  cudaStream_t stream) {
+                  cudaStream_t stream, cudaEvent_t ev_start, cudaEvent_t ev_stop) {
   CUtensorMap mq, mk, mv, mdo;
   fa_status st;
   if ((st = map_bnhd(&mq, q, B, N, H, d)) != FA_OK) return st;
@@ -216,11 +216,16 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   if (d == 64) fa::bwd_pre_kernel<64><<<pre_blocks, 256, 0, stream>>>(p);
   else fa::bwd_pre_kernel<128><<<pre_blocks, 256, 0, stream>>>(p);
   if ((st = check_launch("fa_bwd preprocess launch")) != FA_OK) return st;
+  cudaError_t e;
+  if (ev_start && (e = cudaEventRecord(ev_start, stream)) != cudaSuccess)
+    return cuda_fail(e, "fa_bwd_profiled: record start event");
   if (d == 64) st = causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, p, dev, stream)
                            : launch_bwd_main<64, false>(mq, mk, mv, mdo, p, dev, stream);
   else st = causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, p, dev, stream)
                    : launch_bwd_main<128, false>(mq, mk, mv, mdo, p, dev, stream);
   if (st != FA_OK) return st;
+  if (ev_stop && (e = cudaEventRecord(ev_stop, stream)) != cudaSuccess)
+    return cuda_fail(e, "fa_bwd_profiled: record stop event");
   const long long cv_threads = static_cast<long long>(B) * N * H * tpr;
   const unsigned cv_blocks = static_cast<unsigned>((cv_threads + 255) / 256);
   if (d == 64) fa::bwd_dq_convert_kernel<64><<<cv_blocks, 256, 0, stream>>>(p);
@@ -319,9 +324,11 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
   return fa::bwd_ws_layout(B, H, N, d).total;
 }
 
-fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
-                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const void* out,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int H, int N, int d, int causal, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream, void* main_start,
+                          void* main_stop) {
   if (B < 0 || H < 0 || N < 0) return fail(FA_ERR_INVALID_ARG, "fa_bwd: negative size B=%d H=%d N=%d", B, H, N);
   if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "fa_bwd: head dim %d not supported (64 or 128)", d);
   if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "fa_bwd: scale must be finite");
@@ -343,7 +350,15 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
   fa_status st = current_device(&dev, nullptr);
   if (st != FA_OK) return st;
   return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, N, d, causal != 0, scale, workspace, ws,
-                 dev, static_cast<cudaStream_t>(stream));
+                 dev, static_cast<cudaStream_t>(stream),
+                 static_cast<cudaEvent_t>(main_start), static_cast<cudaEvent_t>(main_stop));
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
+                 int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return fa_bwd_profiled(q, k, v, out, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
+                         workspace_bytes, stream, nullptr, nullptr);
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Ncap, int d) {

@@ -38,6 +38,10 @@ _SIGNATURES = {
     "fa_bwd": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                         _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
                         _c_float, _c_void_p, _c_size_t, _c_void_p]),
+    "fa_bwd_profiled": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                 _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
+                                 _c_int, _c_int, _c_int, _c_float, _c_void_p, _c_size_t,
+                                 _c_void_p, _c_void_p, _c_void_p]),
     "fa_decode_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
     "fa_decode": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                            _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -143,8 +147,12 @@ def bwd_workspace_size(B: int, H: int, N: int, d: int) -> int:
 
 
 def bwd(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = None,
-        dq=None, dk=None, dv=None, workspace=None, stream=None):
-    """Attention backward by recomputation. Returns (dq, dk, dv), bf16 [B, N, H, d]."""
+        dq=None, dk=None, dv=None, workspace=None, stream=None, main_events=None):
+    """Attention backward by recomputation. Returns (dq, dk, dv), bf16 [B, N, H, d].
+
+    main_events: optional (start, stop) torch.cuda.Event pair recorded around the main
+    backward kernel (fa_bwd_profiled), for timing that kernel on its own stream.
+    """
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
         _require(t, name)
         if t.shape != q.shape:
@@ -163,9 +171,18 @@ def bwd(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = 
     if workspace is None:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
     with torch.cuda.device(q.device):
-        _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
-                          _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
-                          _scale(scale, d), _ptr(workspace), workspace.numel(), _stream(stream)))
+        if main_events is None:
+            _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                              _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
+                              _scale(scale, d), _ptr(workspace), workspace.numel(),
+                              _stream(stream)))
+        else:
+            ev0, ev1 = main_events
+            _check(lib.fa_bwd_profiled(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
+                                       _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d,
+                                       int(bool(causal)), _scale(scale, d), _ptr(workspace),
+                                       workspace.numel(), _stream(stream),
+                                       ctypes.c_void_p(ev0.cuda_event), ctypes.c_void_p(ev1.cuda_event)))
     return dq, dk, dv
 
 

@@ -87,6 +87,20 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
                  int causal, float scale, void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * fa_bwd with the same arguments, plus two optional CUDA events (cudaEvent_t, either
+ * may be NULL) that are recorded on `stream` immediately before and immediately after
+ * the main backward kernel (the one that recomputes P and runs the five tile
+ * products). A caller can then time that kernel alone with cudaEventElapsedTime
+ * while the whole backward still runs as one call. Events are not created,
+ * synchronised or destroyed by the library.
+ */
+fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const void* out,
+                          const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                          int H, int N, int d, int causal, float scale, void* workspace,
+                          size_t workspace_bytes, void* stream, void* main_start,
+                          void* main_stop);
+
 /* Bytes of device workspace fa_decode needs (split partials); may be 0. Depends on
  * the current device's SM count, so query it on the device that will run. */
 size_t fa_decode_workspace_size(int B, int H, int Ncap, int d);

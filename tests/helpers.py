@@ -3,7 +3,8 @@ tolerances the tests enforce.
 
 Tolerances (stated for bf16 inputs against the float64 oracle):
   forward  max |out - ref| <= 2e-2 and max |lse - ref| <= 1e-3 (absolute);
-  gradients max |g - ref| <= 5e-2 * max |ref|, per tensor.
+  gradients max |g - ref| <= 5e-2 * max |ref|, per tensor; where the oracle's
+  gradient is identically zero, max |g| <= 1e-5.
 """
 import math
 
@@ -16,6 +17,7 @@ from exact_attention_155_b200.inputs import attention_inputs, to_f64
 OUT_ATOL = 2e-2
 LSE_ATOL = 1e-3
 GRAD_REL = 5e-2
+ZERO_GRAD_ATOL = 1e-5  # for gradients that are exactly zero in the oracle
 
 
 def make_inputs(B, N, H, d, seed, q_mult=1.0, with_dout=True):
@@ -53,8 +55,16 @@ def check_grads(grads, inp, causal, scale, heads=None):
         assert m.any()
         assert np.isfinite(got[m]).all(), name
         err = np.max(np.abs(got[m] - r[m]))
-        bound = GRAD_REL * max(np.max(np.abs(r[m])), 1e-30)
-        errs[name] = err / max(np.max(np.abs(r[m])), 1e-30)
+        ref_max = np.max(np.abs(r[m]))
+        if ref_max == 0.0:
+            # The gradient vanishes identically (e.g. dq with a single visible key:
+            # dS = P (dP - D) = 0). The relative bound is then empty; require the
+            # cancellation to come out at fp32 rounding level instead.
+            assert err <= ZERO_GRAD_ATOL, f"{name}: exact-zero gradient, got max |g| = {err}"
+            errs[name] = err
+            continue
+        bound = GRAD_REL * ref_max
+        errs[name] = err / ref_max
         assert err <= bound, f"{name}: max |d| = {err} > {bound}"
     return errs
 
