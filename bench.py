@@ -277,6 +277,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.synchronize()
     K = args.steps
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    for e in evs:  # create the event handles (torch does so on first record)
+        for x in e:
+            x.record()
     sampler = ClockSampler(local_rank)
     barrier()
     sampler.start()

@@ -274,15 +274,14 @@ __global__ void __launch_bounds__(320, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, 0, 1);   // dV (A in TMEM), dK (A K-major)
-      constexpr uint32_t kIdQ = idesc_bf16_f32(128, D, 1, 1);    // dQ (A MN-major)
-      bool ok = wait_bar(BAR(L::kKVFull), 0, abort_flag, kSiteBwdMma);
-      for (int n = 0; n < niter && ok; ++n) {
-        const int s = n % L::kStages;
-        const uint32_t sQ = base + L::kStage0 + s * L::kStageBytes;
-        const uint32_t sdO = sQ + L::kTile;
-        if (!(ok = wait_bar(BAR(L::kStFull + s), (n / L::kStages) & 1, abort_flag, kSiteBwdMma))) break;
-        tc_fence_after();
-        // S^T = K Q_i^T
+      // d = 128: dQ^T = K^T dS^T (head dim on TMEM lanes, coalesced reductions);
+      // d = 64:  dQ = dS K (queries on TMEM lanes).
+      constexpr uint32_t kIdQ = (D == 128) ? idesc_bf16_f32(128, 128, 1, 1) : idesc_bf16_f32(128, D, 1, 1);
+      auto stage_addr = [&](int n) {
+        return base + L::kStage0 + static_cast<uint32_t>(n % L::kStages) * L::kStageBytes;
+      };
+      auto issue_st = [&](int n) {  // S^T = K Q_n^T
+        const uint32_t sQ = stage_addr(n);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
@@ -290,7 +289,29 @@ __global__ void __launch_bounds__(320, 1)
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(BAR(L::kSFull));
-        // dP^T = V dO_i^T into the region dQ_{i-1} used: wait until it was drained.
+      };
+      bool ok = wait_bar(BAR(L::kKVFull), 0, abort_flag, kSiteBwdMma);
+      if (ok && niter > 0) {
+        ok = wait_bar(BAR(L::kStFull + 0), 0, abort_flag, kSiteBwdMma);
+        if (ok) {
+          tc_fence_after();
+          issue_st(0);
+        }
+      }
+      // Issue order per query tile n: dV(n), dP^T(n), [S^T(n+1)], dK(n), dQ(n), so the
+      // exponentials of tile n+1 overlap the dK/dQ products of tile n.
+      for (int n = 0; n < niter && ok; ++n) {
+        const int s = n % L::kStages;
+        const uint32_t sQ = stage_addr(n);
+        const uint32_t sdO = sQ + L::kTile;
+        // dV += P^T dO_n
+        if (!(ok = wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
+                  (n > 0 || kk > 0) ? 1u : 0u);
+        // dP^T = V dO_n^T, into the region dQ(n-1) used once it has been drained.
         if (n > 0) {
           if (!(ok = wait_bar(BAR(L::kDQFree), (n - 1) & 1, abort_flag, kSiteBwdMma))) break;
           tc_fence_after();
@@ -302,24 +323,31 @@ __global__ void __launch_bounds__(320, 1)
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(BAR(L::kDPFull));
-        // dV += P^T dO_i
-        if (!(ok = wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
-                  (n > 0 || kk > 0) ? 1u : 0u);
-        // dK += dS^T Q_i ; dQ_i = dS K
         if (!(ok = wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma))) break;
         tc_fence_after();
+        // S^T(n+1): the S region is free (P(n) was read by dV(n) and by the dS pass).
+        if (n + 1 < niter) {
+          if (!(ok = wait_bar(BAR(L::kStFull + (n + 1) % L::kStages), ((n + 1) / L::kStages) & 1,
+                              abort_flag, kSiteBwdMma)))
+            break;
+          tc_fence_after();
+          issue_st(n + 1);
+        }
+        // dK += dS^T Q_n
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ss(tDK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
                   sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdKV, (n > 0 || kk > 0) ? 1u : 0u);
+        // dQ_n
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tDQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
-                  sdesc_sw128(sK + kk * 2048, 16384, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk) {
+          if constexpr (D == 128)
+            umma_ss(tDQ, sdesc_sw128(sK + kk * 2048, 16384, 1024),
+                    sdesc_sw128(sDS + kk * 2048, 16384, 1024), kIdQ, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(tDQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                    sdesc_sw128(sK + kk * 2048, 16384, 1024), kIdQ, kk > 0 ? 1u : 0u);
+        }
         umma_commit(BAR(L::kDQFull));
         umma_commit(BAR(L::kDSFree));
         umma_commit(BAR(L::kStEmpty + s));
@@ -445,29 +473,50 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
   } else {
-    // ------------------------------------------- dQ drain (one query per thread)
+    // ------------------------------------------------------------- dQ drain
+    // d = 128: TMEM holds dQ^T (lane = head-dim index j, column = query), so one warp
+    // instruction reduces 32 consecutive floats of one dQ row (128 contiguous bytes).
+    // d = 64: TMEM holds dQ (lane = query), one thread reduces its own row.
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float sc = p.scale;
     for (int n = 0; n < niter; ++n) {
       const int it = it0 + n;
       const bool ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDQFull), n & 1, abort_flag, kSiteBwdDrain));
       if (!ok) break;
       tc_fence_after();
-      const int qrow = it * 128 + r;
-      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Np + qrow) * D;
+      if constexpr (D == 128) {
+        float* col = p.dq_acc + static_cast<size_t>(bh) * p.Np * D + r;
+        const int nq = min(128, p.N - it * 128);  // valid query rows of this tile
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tDQ + lane_off + cc * 32, o);
-        tmem_wait_ld();
-        reg_fence32(o);
-        if (qrow < p.N) {
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tDQ + lane_off + cc * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
-            red_add_v4(dst + cc * 32 + 4 * v, __uint_as_float(o[4 * v]) * p.scale,
-                       __uint_as_float(o[4 * v + 1]) * p.scale, __uint_as_float(o[4 * v + 2]) * p.scale,
-                       __uint_as_float(o[4 * v + 3]) * p.scale);
+          for (int i = 0; i < 32; ++i) {
+            const int qi = cc * 32 + i;
+            if (qi < nq) red_add_f32(col + static_cast<size_t>(it * 128 + qi) * D, __uint_as_float(o[i]) * sc);
+          }
+        }
+      } else {
+        const int qrow = it * 128 + r;
+        float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Np + qrow) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tDQ + lane_off + cc * 32, o);
+          tmem_wait_ld();
+          reg_fence32(o);
+          if (qrow < p.N) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              red_add_v4(dst + cc * 32 + 4 * v, __uint_as_float(o[4 * v]) * sc,
+                         __uint_as_float(o[4 * v + 1]) * sc, __uint_as_float(o[4 * v + 2]) * sc,
+                         __uint_as_float(o[4 * v + 3]) * sc);
+          }
         }
       }
       tc_fence_before();

@@ -273,32 +273,74 @@ __global__ void __launch_bounds__(320, 1)
       float x[128];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(s0[c]) * sl2;
-        x[32 + c] = __uint_as_float(s1[c]) * sl2;
-        x[64 + c] = __uint_as_float(s2[c]) * sl2;
-        x[96 + c] = __uint_as_float(s3[c]) * sl2;
+        x[c] = __uint_as_float(s0[c]);
+        x[32 + c] = __uint_as_float(s1[c]);
+        x[64 + c] = __uint_as_float(s2[c]);
+        x[96 + c] = __uint_as_float(s3[c]);
       }
       const int kbase = j * 128;
-      if (j == diag_j || kbase + 128 > p.N) {
+      const bool masked = (j == diag_j) || (kbase + 128 > p.N);
+      float mx;
+      if (masked) {
+        // Diagonal or tail tile: scale first, then mask to -inf.
         const int lim = CAUSAL ? min(row_g, p.N - 1) : p.N - 1;
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (kbase + c > lim) x[c] = -INFINITY;
-      }
-      float mx = x[0];
+        for (int c = 0; c < 128; ++c) x[c] = (kbase + c > lim) ? -INFINITY : x[c] * sl2;
+        mx = x[0];
 #pragma unroll
-      for (int c = 1; c < 128; ++c) mx = fmaxf(mx, x[c]);
+        for (int c = 1; c < 127; c += 2) mx = max3f(mx, x[c], x[c + 1]);
+        mx = fmaxf(mx, x[127]);
+      } else if (sl2 >= 0.f) {
+        mx = x[0];
+#pragma unroll
+        for (int c = 1; c < 127; c += 2) mx = max3f(mx, x[c], x[c + 1]);
+        mx = fmaxf(mx, x[127]) * sl2;
+      } else {
+        mx = x[0];
+#pragma unroll
+        for (int c = 1; c < 127; c += 2) mx = min3f(mx, x[c], x[c + 1]);
+        mx = fminf(mx, x[127]) * sl2;
+      }
+      // The reference max m moves only when a row's max exceeds it by more than
+      // 2^8 (log2 units): until then p = 2^(x - m) <= 256, which fp32 and bf16 hold
+      // exactly enough, and O / l stays exact because both use the same m.
       const float m_new = fmaxf(m, mx);
-      const float ms = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ex2_approx(m - ms);
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ex2_approx(x[c] - ms);
-        rs += x[c];
+      const bool rescale = __any_sync(0xffffffffu, m_new > m + 8.f);
+      float alpha = 1.f;
+      if (rescale) {
+        alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf)
+        l *= alpha;
+        m = m_new;
       }
-      if (j > 0 && __any_sync(0xffffffffu, m_new > m)) {
-        // The running max grew: rescale this row's partial output in TMEM.
+      const float ms = (m == -INFINITY) ? 0.f : m;
+      const float nms = -ms;
+      float rs0 = 0.f, rs1 = 0.f;
+      // p = 2^(x - m), row sum, bf16 pack, and store to TMEM 32 columns at a time so
+      // the packed words never coexist with the whole fp32 row.
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int c = ch * 32 + 2 * i;
+          float a = x[c], bb = x[c + 1];
+          if (masked) {
+            a -= ms;
+            bb -= ms;
+          } else {
+            fma2(a, bb, a, bb, sl2, sl2, nms, nms);
+          }
+          a = ex2_approx(a);
+          bb = ex2_approx(bb);
+          add2(rs0, rs1, rs0, rs1, a, bb);
+          pk[i] = pack_bf16x2(a, bb);
+        }
+        tmem_st16(tS + ch * 16, pk);
+      }
+      l += rs0 + rs1;
+      if (rescale && j > 0) {
+        // Rescale this row's partial output in TMEM; PV for this tile is issued only
+        // after the arrive below, so O is stable (S_t(j) was committed after PV_t(j-1)).
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -306,20 +348,15 @@ __global__ void __launch_bounds__(320, 1)
           tmem_wait_ld();
           reg_fence32(o);
 #pragma unroll
-          for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+          for (int c = 0; c < 32; c += 2) {
+            float a0, a1;
+            mul2(a0, a1, __uint_as_float(o[c]), __uint_as_float(o[c + 1]), alpha, alpha);
+            o[c] = __float_as_uint(a0);
+            o[c + 1] = __float_as_uint(a1);
+          }
           tmem_st32(tO + cc * 32, o);
         }
       }
-      l = l * alpha + rs;
-      m = m_new;
-      uint32_t pk0[32], pk1[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        pk0[c] = pack_bf16x2(x[2 * c], x[2 * c + 1]);
-        pk1[c] = pack_bf16x2(x[64 + 2 * c], x[64 + 2 * c + 1]);
-      }
-      tmem_st32(tS + 0, pk0);
-      tmem_st32(tS + 32, pk1);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(L::kPFull + t));

@@ -178,6 +178,9 @@ def bwd(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = 
                               _stream(stream)))
         else:
             ev0, ev1 = main_events
+            for ev in (ev0, ev1):
+                if ev.cuda_event == 0:
+                    ev.record()  # torch creates the CUDA event handle lazily
             _check(lib.fa_bwd_profiled(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout),
                                        _ptr(lse), _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d,
                                        int(bool(causal)), _scale(scale, d), _ptr(workspace),
