@@ -127,18 +127,22 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const BwdParams p) 
 template <int D>
 struct BwdLayout {
   static constexpr int kTile = 128 * D * 2;  // one 128-row bf16 tile
-  static constexpr int kStages = (D == 128) ? 2 : 3;
+  static constexpr int kQStages = 2;         // Q_i (+ lse2_i, D_i) double-buffered
   static constexpr int kK = 0;
   static constexpr int kV = kTile;
-  static constexpr int kStage0 = 2 * kTile;  // stage s: Q at +0, dO at +kTile
-  static constexpr int kStageBytes = 2 * kTile;
-  static constexpr int kDS = kStage0 + kStages * kStageBytes;  // 128 x 128 bf16 dS^T
-  static constexpr int kVec = kDS + 32768;                     // per stage: lse2[128], D[128]
-  static constexpr int kBar = kVec + kStages * 1024;
+  static constexpr int kQ0 = 2 * kTile;                      // kQStages tiles
+  static constexpr int kDO = kQ0 + kQStages * kTile;         // dO_i, single buffer
+  static constexpr int kDS = kDO + kTile;                    // 128 x 128 bf16 dS^T
+  static constexpr int kStage = kDS + 32768;                 // 2 x 16 KB dQ staging (d = 128)
+  static constexpr int kStageBytes = (D == 128) ? 2 * 16384 : 0;
+  static constexpr int kVec = kStage + kStageBytes;          // per Q stage: lse2[128], D[128]
+  static constexpr int kBar = kVec + kQStages * 1024;
   static constexpr int kKVFull = 0;
-  static constexpr int kStFull = 1;                  // [kStages]
-  static constexpr int kStEmpty = 1 + kStages;       // [kStages]
-  static constexpr int kSFull = 1 + 2 * kStages;
+  static constexpr int kQFull = 1;                   // [kQStages]
+  static constexpr int kQEmpty = 1 + kQStages;       // [kQStages]
+  static constexpr int kDOFull = 1 + 2 * kQStages;
+  static constexpr int kDOEmpty = kDOFull + 1;
+  static constexpr int kSFull = kDOFull + 2;
   static constexpr int kDPFull = kSFull + 1;
   static constexpr int kPFull = kSFull + 2;
   static constexpr int kDSFull = kSFull + 3;
@@ -174,6 +178,35 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                "f"(d)
                : "memory");
 }
+__device__ __forceinline__ void bulk_reduce_add_f32(float* gdst, uint32_t ssrc, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst),
+               "r"(ssrc), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read1() {
+  asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+// Barrier over `nthreads` threads that also returns the AND of every thread's predicate.
+__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %1, 0;\n\t"
+      "bar.red.and.pred po, %2, %3, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
@@ -208,10 +241,12 @@ __global__ void __launch_bounds__(320, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(L::kKVFull), 1);
-    for (int s = 0; s < L::kStages; ++s) {
-      mbar_init(BAR(L::kStFull + s), 1);
-      mbar_init(BAR(L::kStEmpty + s), 1);
+    for (int s = 0; s < L::kQStages; ++s) {
+      mbar_init(BAR(L::kQFull + s), 1);
+      mbar_init(BAR(L::kQEmpty + s), 1);
     }
+    mbar_init(BAR(L::kDOFull), 1);
+    mbar_init(BAR(L::kDOEmpty), 1);
     mbar_init(BAR(L::kSFull), 1);
     mbar_init(BAR(L::kDPFull), 1);
     mbar_init(BAR(L::kPFull), 128);
@@ -249,24 +284,30 @@ __global__ void __launch_bounds__(320, 1)
       }
       const float* lse2_h = p.lse2 + static_cast<size_t>(bh) * p.Np;
       const float* dvec_h = p.dvec + static_cast<size_t>(bh) * p.Np;
-      int n = 0;
-      for (; n < niter; ++n) {
+      int nq = 0, ndo = 0;  // loads issued
+      for (int n = 0; n < niter; ++n) {
         const int it = it0 + n;
-        const int s = n % L::kStages;
-        if (!wait_bar(BAR(L::kStEmpty + s), ((n / L::kStages) & 1) ^ 1u, abort_flag, kSiteBwdProducer))
+        const int s = n % L::kQStages;
+        if (!wait_bar(BAR(L::kQEmpty + s), ((n / L::kQStages) & 1) ^ 1u, abort_flag, kSiteBwdProducer))
           break;
-        const uint32_t st = base + L::kStage0 + s * L::kStageBytes;
-        mbar_arrive_expect_tx(BAR(L::kStFull + s), 2 * L::kTile + 1024);
-        for (int bx = 0; bx < D / 64; ++bx) {
-          tma_load_4d(st + bx * 16384, &tmQ, BAR(L::kStFull + s), bx * 64, h, it * 128, b);
-          tma_load_4d(st + L::kTile + bx * 16384, &tmdO, BAR(L::kStFull + s), bx * 64, h, it * 128, b);
-        }
+        const uint32_t sQ = base + L::kQ0 + s * L::kTile;
+        mbar_arrive_expect_tx(BAR(L::kQFull + s), L::kTile + 1024);
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_4d(sQ + bx * 16384, &tmQ, BAR(L::kQFull + s), bx * 64, h, it * 128, b);
         const uint32_t sv = base + L::kVec + s * 1024;
-        bulk_load(sv, lse2_h + it * 128, 512, BAR(L::kStFull + s));
-        bulk_load(sv + 512, dvec_h + it * 128, 512, BAR(L::kStFull + s));
+        bulk_load(sv, lse2_h + it * 128, 512, BAR(L::kQFull + s));
+        bulk_load(sv + 512, dvec_h + it * 128, 512, BAR(L::kQFull + s));
+        ++nq;
+        if (!wait_bar(BAR(L::kDOEmpty), (n & 1) ^ 1u, abort_flag, kSiteBwdProducer)) break;
+        mbar_arrive_expect_tx(BAR(L::kDOFull), L::kTile);
+        for (int bx = 0; bx < D / 64; ++bx)
+          tma_load_4d(base + L::kDO + bx * 16384, &tmdO, BAR(L::kDOFull), bx * 64, h, it * 128, b);
+        ++ndo;
       }
-      for (int k = max(0, n - L::kStages); k < n; ++k)
-        drain_wait(BAR(L::kStFull + k % L::kStages), (k / L::kStages) & 1);
+      // Never leave the CTA with copies in flight.
+      for (int k = max(0, nq - L::kQStages); k < nq; ++k)
+        drain_wait(BAR(L::kQFull + k % L::kQStages), (k / L::kQStages) & 1);
+      if (ndo > 0) drain_wait(BAR(L::kDOFull), (ndo - 1) & 1);
       drain_wait(BAR(L::kKVFull), 0);
     }
   } else if (warp == 9) {
@@ -277,11 +318,10 @@ __global__ void __launch_bounds__(320, 1)
       // d = 128: dQ^T = K^T dS^T (head dim on TMEM lanes, coalesced reductions);
       // d = 64:  dQ = dS K (queries on TMEM lanes).
       constexpr uint32_t kIdQ = (D == 128) ? idesc_bf16_f32(128, 128, 1, 1) : idesc_bf16_f32(128, D, 1, 1);
-      auto stage_addr = [&](int n) {
-        return base + L::kStage0 + static_cast<uint32_t>(n % L::kStages) * L::kStageBytes;
-      };
+      auto q_addr = [&](int n) { return base + L::kQ0 + static_cast<uint32_t>(n % L::kQStages) * L::kTile; };
+      const uint32_t sdO = base + L::kDO;
       auto issue_st = [&](int n) {  // S^T = K Q_n^T
-        const uint32_t sQ = stage_addr(n);
+        const uint32_t sQ = q_addr(n);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
@@ -292,26 +332,26 @@ __global__ void __launch_bounds__(320, 1)
       };
       bool ok = wait_bar(BAR(L::kKVFull), 0, abort_flag, kSiteBwdMma);
       if (ok && niter > 0) {
-        ok = wait_bar(BAR(L::kStFull + 0), 0, abort_flag, kSiteBwdMma);
+        ok = wait_bar(BAR(L::kQFull + 0), 0, abort_flag, kSiteBwdMma);
         if (ok) {
           tc_fence_after();
           issue_st(0);
         }
       }
-      // Issue order per query tile n: dV(n), dP^T(n), [S^T(n+1)], dK(n), dQ(n), so the
+      // Issue order per query tile n: dV(n), dP^T(n), [S^T(n+1)], dK(n), dQ(n): the
       // exponentials of tile n+1 overlap the dK/dQ products of tile n.
       for (int n = 0; n < niter && ok; ++n) {
-        const int s = n % L::kStages;
-        const uint32_t sQ = stage_addr(n);
-        const uint32_t sdO = sQ + L::kTile;
+        const int s = n % L::kQStages;
+        const uint32_t sQ = q_addr(n);
         // dV += P^T dO_n
         if (!(ok = wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        if (!(ok = wait_bar(BAR(L::kDOFull), n & 1, abort_flag, kSiteBwdMma))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ts(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
                   (n > 0 || kk > 0) ? 1u : 0u);
-        // dP^T = V dO_n^T, into the region dQ(n-1) used once it has been drained.
+        // dP^T = V dO_n^T, into the columns dQ(n-1) used once they were read out.
         if (n > 0) {
           if (!(ok = wait_bar(BAR(L::kDQFree), (n - 1) & 1, abort_flag, kSiteBwdMma))) break;
           tc_fence_after();
@@ -323,11 +363,12 @@ __global__ void __launch_bounds__(320, 1)
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(BAR(L::kDPFull));
+        umma_commit(BAR(L::kDOEmpty));
         if (!(ok = wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma))) break;
         tc_fence_after();
-        // S^T(n+1): the S region is free (P(n) was read by dV(n) and by the dS pass).
+        // S^T(n+1): the S columns are free (P(n) was read by dV(n); the dS pass is done).
         if (n + 1 < niter) {
-          if (!(ok = wait_bar(BAR(L::kStFull + (n + 1) % L::kStages), ((n + 1) / L::kStages) & 1,
+          if (!(ok = wait_bar(BAR(L::kQFull + (n + 1) % L::kQStages), ((n + 1) / L::kQStages) & 1,
                               abort_flag, kSiteBwdMma)))
             break;
           tc_fence_after();
@@ -350,7 +391,7 @@ __global__ void __launch_bounds__(320, 1)
         }
         umma_commit(BAR(L::kDQFull));
         umma_commit(BAR(L::kDSFree));
-        umma_commit(BAR(L::kStEmpty + s));
+        umma_commit(BAR(L::kQEmpty + s));
       }
       if (ok) umma_commit(BAR(L::kMmaDone));
       umma_commit(BAR(L::kDrain));
@@ -366,10 +407,10 @@ __global__ void __launch_bounds__(320, 1)
     bool ok = true;
     for (int n = 0; n < niter; ++n) {
       const int it = it0 + n;
-      const int s = n % L::kStages;
+      const int s = n % L::kQStages;
       const float* vec = reinterpret_cast<const float*>(smem + L::kVec + s * 1024);
       ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kSFull), n & 1, abort_flag, kSiteBwdSoftmax));
-      if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kStFull + s), (n / L::kStages) & 1,
+      if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kQFull + s), (n / L::kQStages) & 1,
                                                    abort_flag, kSiteBwdSoftmax));
       if (!ok) break;
       tc_fence_after();
@@ -483,24 +524,46 @@ __global__ void __launch_bounds__(320, 1)
     const float sc = p.scale;
     for (int n = 0; n < niter; ++n) {
       const int it = it0 + n;
-      const bool ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDQFull), n & 1, abort_flag, kSiteBwdDrain));
+      bool ok = wait_bar(BAR(L::kDQFull), n & 1, abort_flag, kSiteBwdDrain);
+      // All four drain warps leave together: they share named barriers below.
+      ok = named_bar_and(1, 128, ok);
       if (!ok) break;
       tc_fence_after();
       if constexpr (D == 128) {
-        float* col = p.dq_acc + static_cast<size_t>(bh) * p.Np * D + r;
-        const int nq = min(128, p.N - it * 128);  // valid query rows of this tile
+        // Read all of dQ^T (128 queries for this thread's head-dim index r), free the
+        // TMEM columns, then push 32-query chunks through shared memory with one
+        // asynchronous 16 KB bulk reduction each (rows of the accumulator are
+        // contiguous: [bh][query][d]).
+        uint32_t o0[32], o1[32], o2[32], o3[32];
+        tmem_ld32(tDQ + lane_off + 0, o0);
+        tmem_ld32(tDQ + lane_off + 32, o1);
+        tmem_ld32(tDQ + lane_off + 64, o2);
+        tmem_ld32(tDQ + lane_off + 96, o3);
+        tmem_wait_ld();
+        reg_fence32(o0);
+        reg_fence32(o1);
+        reg_fence32(o2);
+        reg_fence32(o3);
+        tc_fence_before();
+        mbar_arrive(BAR(L::kDQFree));
+        float* gtile = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(it) * 128) * D;
+        const bool leader = (warp == 4 && lane == 0);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tDQ + lane_off + cc * 32, o);
-          tmem_wait_ld();
-          reg_fence32(o);
+          const uint32_t buf = base + L::kStage + (cc & 1) * 16384;
+          if (leader) bulk_wait_read1();  // the reduction that used this buffer has read it
+          named_bar_sync(1, 128);
+          const uint32_t* src = cc == 0 ? o0 : (cc == 1 ? o1 : (cc == 2 ? o2 : o3));
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int qi = cc * 32 + i;
-            if (qi < nq) red_add_f32(col + static_cast<size_t>(it * 128 + qi) * D, __uint_as_float(o[i]) * sc);
+          for (int i = 0; i < 32; ++i) st_shared_f32(buf + (i * 128 + r) * 4, __uint_as_float(src[i]) * sc);
+          fence_proxy_async_smem();
+          named_bar_sync(1, 128);
+          if (leader) {
+            bulk_reduce_add_f32(gtile + cc * 32 * D, buf, 16384);
+            bulk_commit();
           }
         }
+        continue;
       } else {
         const int qrow = it * 128 + r;
         float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Np + qrow) * D;
@@ -521,6 +584,9 @@ __global__ void __launch_bounds__(320, 1)
       }
       tc_fence_before();
       mbar_arrive(BAR(L::kDQFree));
+    }
+    if constexpr (D == 128) {
+      if (warp == 4 && lane == 0) bulk_wait_all();  // reductions complete before exit
     }
   }
 
