@@ -393,6 +393,18 @@ def run_ours(args, rank, world, local_rank):
                           workspace=ws5)
         steps100()
         sms = timed_events(torch, steps100, 5)
+        # The same 100 steps replayed from one CUDA graph: no host launch overhead.
+        graph = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            steps100()
+        torch.cuda.current_stream().wait_stream(side)
+        with torch.cuda.graph(graph):
+            steps100()
+        graph.replay()
+        gms = timed_events(torch, graph.replay, 10)
+        del graph
         parts = {
             "prefill_fwd": {"workload": "causal fwd B=1 H=32 N=8192 d=128", "value": ptf,
                             "unit": "TFLOP/s", "ms": pms, "roofline_bound": "tensor",
@@ -408,6 +420,7 @@ def run_ours(args, rank, world, local_rank):
                              "l2": "flushed (512 MiB write) before every call"},
             "decode_steps": {"workload": "decode B=2 H=16 d=64 cap 2048, 100 appending steps",
                              "us_per_step": sms * 1e3 / c5["steps"],
+                             "us_per_step_cuda_graph": gms * 1e3 / c5["steps"],
                              "gb_s": 8192 * sum(t + 1 for t in range(c5["steps"]))
                              / (sms * 1e-3) / 1e9},
         }

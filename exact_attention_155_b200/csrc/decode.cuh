@@ -4,26 +4,30 @@
 // 推理优化与KV缓存 of "FlashAttention与MindSpore 2.0全场景融合方案").
 //
 // The work is a matrix-vector product per head, bound by reading K and V once from
-// HBM, so it runs on CUDA cores (no tensor-core reshaping):
-//  * decode_split_kernel: grid (splits, H, B). Each CTA takes one contiguous chunk
-//    of keys, reads each K and V row once with 16-byte coalesced loads (d/8 lanes
-//    per row, several rows in flight per thread), keeps the chunk's scores in
-//    shared memory, and writes a partial (o_s, lse_s) for its chunk. The CTA whose
-//    chunk holds the appended row writes that row into the cache and uses k_new /
-//    v_new directly, so no other CTA reads it.
-//  * decode_merge_kernel: LSE = log sum_s exp(lse_s), O = sum_s exp(lse_s - LSE) o_s,
-//    the stable combination of per-block (m, l) of the blockwise softmax (section
-//    2.2.2 of "FlashAttention优化Transformer显存与计算效率").
-// With a single split the split kernel writes the final bf16 output itself.
+// HBM, so it runs on CUDA cores (no tensor-core reshaping). decode_kernel: grid
+// (splits, H, B) where the `splits` CTAs of one (batch, head) form a thread-block
+// cluster. Each CTA takes one contiguous chunk of keys; d/8 lanes share a cache row
+// (16-byte coalesced loads), K and V rows of several steps are loaded together,
+// and each lane group keeps a running (m, l, o) online-softmax state, so a step has
+// no block-wide synchronisation. Warp states are combined with shuffles, CTA states
+// in shared memory, and the cluster's CTA states in the leader CTA's shared memory
+// (the stable combination of per-block (m, l) of section 2.2.2 of
+// "FlashAttention优化Transformer显存与计算效率"). The CTA whose chunk holds the
+// appended row writes that row into the cache and every CTA reads it from k_new /
+// v_new, so no CTA reads a row another one writes.
 #pragma once
 
 #include <math.h>
+
+#include <cooperative_groups.h>
 
 #include "ptx.cuh"
 
 namespace fa {
 
-constexpr int kDecodeMaxChunk = 2048;  // keys per split (scores live in shared memory)
+namespace cg = cooperative_groups;
+
+constexpr int kDecodeMaxSplits = 8;  // CTAs per (batch, head): one portable cluster
 
 struct DecodeParams {
   const uint16_t* q;      // [B, 1, H, d]
@@ -34,8 +38,6 @@ struct DecodeParams {
   const uint16_t* v_new;  // [B, 1, H, d] or null
   uint16_t* out;          // [B, 1, H, d]
   float* lse;             // [B, H] or null
-  float* part_o;          // [B, H, nsplit, d] (nsplit > 1)
-  float* part_lse;        // [B, H, nsplit]    (nsplit > 1)
   int B, H, Ncap, nsplit, chunk;
   float scale_log2;
 };
@@ -51,17 +53,37 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   }
 }
 
-template <int D>
-__global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p) {
-  constexpr int LPR = D / 8;     // lanes per cache row (16 bytes each)
-  constexpr int RPW = 32 / LPR;  // rows per warp step
-  constexpr int RPC = 4 * RPW;   // rows per CTA step
-  constexpr int U = 4;           // row steps kept in flight per thread
-  __shared__ float s_sc[kDecodeMaxChunk];
-  __shared__ float s_red[4];
-  __shared__ float s_o[4][D];
+// Running (m, l, o) state of the online softmax: m in log2 units, l = sum 2^(s - m),
+// o = sum 2^(s - m) v (unnormalised). Combining two states rescales both to the
+// larger max (the stable block combination of section 2.2.2).
+__device__ __forceinline__ void online_merge(float& m, float& l, float (&o)[8], float m2, float l2,
+                                             const float (&o2)[8]) {
+  const float mn = fmaxf(m, m2);
+  if (mn == -INFINITY) return;  // both empty
+  const float c1 = (m == -INFINITY) ? 0.f : ex2_approx(m - mn);
+  const float c2 = (m2 == -INFINITY) ? 0.f : ex2_approx(m2 - mn);
+  l = l * c1 + l2 * c2;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = o[i] * c1 + o2[i] * c2;
+  m = mn;
+}
 
-  const int split = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+// One CTA per (split, head, batch); the `splits` CTAs of a (batch, head) form one
+// thread-block cluster and combine their partial states in the leader CTA's shared
+// memory (distributed shared memory), so the whole step is a single launch with no
+// global workspace.
+template <int D>
+__global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
+  constexpr int LPR = D / 8;     // lanes per cache row (16 bytes each)
+  constexpr int RPW = 32 / LPR;  // rows per warp per step
+  constexpr int U = 4;           // steps whose loads are issued together
+  constexpr int RSTEP = 4 * RPW; // rows per CTA per step
+  __shared__ float s_warp[4][D + 2];   // per-warp partial: o[D], m, l
+  __shared__ float s_part[8][D + 2];   // leader only: per-CTA partials of the cluster
+
+  cg::cluster_group cluster = cg::this_cluster();
+  const int split = static_cast<int>(cluster.block_rank());
+  const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int grp = lane / LPR, sub = lane % LPR;
   const bool append = p.k_new != nullptr;
@@ -78,7 +100,6 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
   const int Lt = L + (do_append ? 1 : 0);
   const int k0 = split * p.chunk;
   const int k1 = min(k0 + p.chunk, Lt);
-  const int n = max(0, k1 - k0);
   const size_t bh = static_cast<size_t>(b) * p.H + h;
   const size_t row_stride = static_cast<size_t>(p.H) * D;  // elements between cache rows
   const uint16_t* kc = p.k_cache + (static_cast<size_t>(b) * p.Ncap * p.H + h) * D + sub * 8;
@@ -86,7 +107,8 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
   const uint16_t* kn = append ? p.k_new + bh * D + sub * 8 : nullptr;
   const uint16_t* vn = append ? p.v_new + bh * D + sub * 8 : nullptr;
 
-  // This chunk holds the appended row: persist it in the cache.
+  // The CTA whose chunk holds the appended row persists it in the cache; every CTA
+  // reads that row from k_new / v_new, never from the cache.
   if (do_append && L >= k0 && L < k1 && tid < LPR) {
     const size_t off = (static_cast<size_t>(b) * p.Ncap + L) * row_stride + h * D + tid * 8;
     *reinterpret_cast<uint4*>(p.k_cache + off) =
@@ -103,18 +125,26 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
     for (int i = 0; i < 8; ++i) qf[i] *= p.scale_log2;
   }
 
-  // Phase 1: scores (log2 units) of this chunk's keys.
-  for (int base = k0 + warp * RPW; base < k1; base += U * RPC) {
-    uint4 kv[U];
+  float m = -INFINITY, l = 0.f, o[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o[i] = 0.f;
+
+  // Rows handled by this lane group: k0 + warp*RPW + grp + RSTEP*t, t = 0, 1, ...
+  for (int base = k0 + warp * RPW; base < k1; base += U * RSTEP) {
+    uint4 kv[U], vv[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int kb = base + u * RPC + grp;
+      const int kb = base + u * RSTEP + grp;
       kv[u] = make_uint4(0, 0, 0, 0);
+      vv[u] = make_uint4(0, 0, 0, 0);
       if (kb < k1) {
-        const uint16_t* src = (do_append && kb == L) ? kn : kc + static_cast<size_t>(kb) * row_stride;
-        kv[u] = __ldg(reinterpret_cast<const uint4*>(src));
+        const bool is_new = do_append && kb == L;
+        const size_t off = static_cast<size_t>(kb) * row_stride;
+        kv[u] = __ldg(reinterpret_cast<const uint4*>(is_new ? kn : kc + off));
+        vv[u] = __ldg(reinterpret_cast<const uint4*>(is_new ? vn : vc + off));
       }
     }
+    float sc[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       float f[8];
@@ -123,109 +153,95 @@ __global__ void __launch_bounds__(128) decode_split_kernel(const DecodeParams p)
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc = fmaf(qf[i], f[i], acc);
 #pragma unroll
-      for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-      const int kb = base + u * RPC + grp;
-      if (sub == 0 && kb < k1) s_sc[kb - k0] = acc;
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      sc[u] = (base + u * RSTEP + grp < k1) ? acc : -INFINITY;
     }
-  }
-  __syncthreads();
-
-  // Phase 2: chunk max and exp-sum.
-  float mx = -INFINITY;
-  for (int i = tid; i < n; i += 128) mx = fmaxf(mx, s_sc[i]);
+    float mx = sc[0];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) s_red[warp] = mx;
-  __syncthreads();
-  const float m = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-  const float ms = (m == -INFINITY) ? 0.f : m;
-  __syncthreads();
-  float sum = 0.f;
-  for (int i = tid; i < n; i += 128) {
-    const float e = ex2_approx(s_sc[i] - ms);
-    s_sc[i] = e;
-    sum += e;
-  }
+    for (int u = 1; u < U; ++u) mx = fmaxf(mx, sc[u]);
+    const float m_new = fmaxf(m, mx);
+    if (m_new != -INFINITY) {
+      const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+      l *= alpha;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-  if (lane == 0) s_red[warp] = sum;
-  __syncthreads();
-  const float l = s_red[0] + s_red[1] + s_red[2] + s_red[3];
-
-  // Phase 3: weighted sum of V rows.
-  float acc[8];
+      for (int i = 0; i < 8; ++i) o[i] *= alpha;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int base = k0 + warp * RPW; base < k1; base += U * RPC) {
-    uint4 vv[U];
+      for (int u = 0; u < U; ++u) {
+        const float pu = ex2_approx(sc[u] - m_new);  // 0 for rows past the chunk
+        float f[8];
+        bf16x8_to_f32(vv[u], f);
+        l += pu;
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int kb = base + u * RPC + grp;
-      vv[u] = make_uint4(0, 0, 0, 0);
-      if (kb < k1) {
-        const uint16_t* src = (do_append && kb == L) ? vn : vc + static_cast<size_t>(kb) * row_stride;
-        vv[u] = __ldg(reinterpret_cast<const uint4*>(src));
+        for (int i = 0; i < 8; ++i) o[i] = fmaf(pu, f[i], o[i]);
       }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      const int kb = base + u * RPC + grp;
-      const float w = (kb < k1) ? s_sc[kb - k0] : 0.f;
-      float f[8];
-      bf16x8_to_f32(vv[u], f);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(w, f[i], acc[i]);
+      m = m_new;
     }
   }
+
+  // Combine the RPW row groups of the warp (lanes with the same slice `sub`).
 #pragma unroll
-  for (int o = LPR; o < 32; o <<= 1)
+  for (int off = LPR; off < 32; off <<= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, off);
+    const float l2 = __shfl_xor_sync(0xffffffffu, l, off);
+    float o2[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    for (int i = 0; i < 8; ++i) o2[i] = __shfl_xor_sync(0xffffffffu, o[i], off);
+    online_merge(m, l, o, m2, l2, o2);
+  }
   if (grp == 0) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) s_o[warp][sub * 8 + i] = acc[i];
+    for (int i = 0; i < 8; ++i) s_warp[warp][sub * 8 + i] = o[i];
+    if (sub == 0) {
+      s_warp[warp][D] = m;
+      s_warp[warp][D + 1] = l;
+    }
   }
   __syncthreads();
 
-  const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-  const float lse_nat = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-  if (p.nsplit == 1) {
-    if (tid < D / 2) {
-      const int c = 2 * tid;
-      const float o0 = (s_o[0][c] + s_o[1][c] + s_o[2][c] + s_o[3][c]) * inv_l;
-      const float o1 = (s_o[0][c + 1] + s_o[1][c + 1] + s_o[2][c + 1] + s_o[3][c + 1]) * inv_l;
-      reinterpret_cast<uint32_t*>(p.out + bh * D)[tid] = pack_bf16x2(o0, o1);
+  // CTA partial -> the leader CTA's shared memory.
+  float* dst = cluster.map_shared_rank(&s_part[0][0], 0) + split * (D + 2);
+  if (tid < D) {
+    float mc = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) mc = fmaxf(mc, s_warp[w][D]);
+    float oc = 0.f, lc = 0.f;
+    if (mc != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float mw = s_warp[w][D];
+        const float cw = (mw == -INFINITY) ? 0.f : ex2_approx(mw - mc);
+        oc = fmaf(s_warp[w][tid], cw, oc);
+        lc = fmaf(s_warp[w][D + 1], cw, lc);
+      }
     }
-    if (tid == 0 && p.lse) p.lse[bh] = lse_nat;
-  } else {
-    if (tid < D) {
-      const float o = (s_o[0][tid] + s_o[1][tid] + s_o[2][tid] + s_o[3][tid]) * inv_l;
-      p.part_o[(bh * p.nsplit + split) * D + tid] = o;
+    dst[tid] = oc;
+    if (tid == 0) {
+      dst[D] = mc;
+      dst[D + 1] = lc;
     }
-    if (tid == 0) p.part_lse[bh * p.nsplit + split] = lse_nat;
   }
-}
+  cluster.sync();
 
-template <int D>
-__global__ void __launch_bounds__(D) decode_merge_kernel(const DecodeParams p) {
-  const size_t bh = blockIdx.x;
-  const int tid = threadIdx.x;
-  const float* pl = p.part_lse + bh * p.nsplit;
-  float m = -INFINITY;
-  for (int s = 0; s < p.nsplit; ++s) m = fmaxf(m, pl[s]);
-  float tot = 0.f, acc = 0.f;
-  if (m != -INFINITY) {
-    for (int s = 0; s < p.nsplit; ++s) {
-      const float w = expf(pl[s] - m);
-      tot += w;
-      acc = fmaf(w, p.part_o[(bh * p.nsplit + s) * D + tid], acc);
+  if (split == 0 && tid < D) {
+    const int S = static_cast<int>(cluster.num_blocks());
+    float M = -INFINITY;
+    for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, s_part[s2][D]);
+    float O = 0.f, Ls = 0.f;
+    if (M != -INFINITY) {
+      for (int s2 = 0; s2 < S; ++s2) {
+        const float ms = s_part[s2][D];
+        const float c = (ms == -INFINITY) ? 0.f : ex2_approx(ms - M);
+        O = fmaf(s_part[s2][tid], c, O);
+        Ls = fmaf(s_part[s2][D + 1], c, Ls);
+      }
     }
+    const float out = (Ls > 0.f) ? O / Ls : 0.f;
+    const float nb = __shfl_down_sync(0xffffffffu, out, 1);
+    if ((tid & 1) == 0)
+      reinterpret_cast<uint32_t*>(p.out + bh * D)[tid >> 1] = pack_bf16x2(out, nb);
+    if (tid == 0 && p.lse)
+      p.lse[bh] = (Ls > 0.f) ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
   }
-  const float o = (tot > 0.f) ? acc / tot : 0.f;
-  const float o_nb = __shfl_down_sync(0xffffffffu, o, 1);
-  if ((tid & 1) == 0)
-    reinterpret_cast<uint32_t*>(p.out + bh * D)[tid >> 1] = pack_bf16x2(o, o_nb);
-  if (tid == 0 && p.lse) p.lse[bh] = (tot > 0.f) ? m + logf(tot) : -INFINITY;
 }
 
 }  // namespace fa

@@ -233,28 +233,16 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   return check_launch("fa_bwd dq convert launch");
 }
 
+// CTAs per (batch, head) for decode: a power of two <= 8 (one portable cluster)
+// so the grid is about one wave (6 CTAs per SM), with at least 64 keys per CTA.
 int decode_splits(int B, int H, int Ncap, int sms, int* chunk_out) {
   const long long heads = static_cast<long long>(B) * H;
-  const int min_split = (Ncap + fa::kDecodeMaxChunk - 1) / fa::kDecodeMaxChunk;
-  const int max_split = std::max(1, (Ncap + 63) / 64);  // at least 64 keys per split
-  long long ns = (static_cast<long long>(sms) * 8 + heads - 1) / std::max(1LL, heads);
-  ns = std::min<long long>(ns, max_split);
-  ns = std::max<long long>(ns, min_split);
-  ns = std::max<long long>(ns, 1);
-  int chunk = static_cast<int>((Ncap + ns - 1) / ns);
-  chunk = (chunk + 15) / 16 * 16;
-  if (chunk > fa::kDecodeMaxChunk) chunk = fa::kDecodeMaxChunk;
-  const int nsplit = (Ncap + chunk - 1) / chunk;
+  const long long want = (static_cast<long long>(sms) * 6 + heads - 1) / std::max(1LL, heads);
+  int ns = 1;
+  while (ns < fa::kDecodeMaxSplits && ns < want && static_cast<long long>(ns) * 2 * 64 <= Ncap) ns *= 2;
+  const int chunk = (Ncap + ns - 1) / ns;
   if (chunk_out) *chunk_out = chunk;
-  return nsplit;
-}
-
-size_t decode_ws_bytes(int B, int H, int d, int nsplit) {
-  if (nsplit <= 1) return 0;
-  const size_t heads = static_cast<size_t>(B) * H;
-  const size_t o_bytes = heads * nsplit * d * sizeof(float);
-  const size_t o_pad = (o_bytes + 255) / 256 * 256;
-  return o_pad + heads * nsplit * sizeof(float);
+  return ns;
 }
 
 __global__ void timeout_probe_kernel(long long limit) {
@@ -362,9 +350,11 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Ncap, int d) {
-  if (B <= 0 || H <= 0 || Ncap <= 0 || (d != 64 && d != 128)) return 0;
-  const int ns = decode_splits(B, H, Ncap, sm_count_or_default(), nullptr);
-  return decode_ws_bytes(B, H, d, ns);
+  (void)B;
+  (void)H;
+  (void)Ncap;
+  (void)d;
+  return 0;  // split partials are combined on chip (cluster shared memory)
 }
 
 fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cache_seqlens,
@@ -391,11 +381,8 @@ fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cach
   if (st != FA_OK) return st;
   int chunk = 0;
   const int ns = decode_splits(B, H, Ncap, sms, &chunk);
-  const size_t need = decode_ws_bytes(B, H, d, ns);
-  if (need > 0 && (!workspace || workspace_bytes < need))
-    return fail(FA_ERR_WORKSPACE, "fa_decode: workspace needs %zu bytes, got %zu", need, workspace_bytes);
-  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
-    return fail(FA_ERR_INVALID_ARG, "fa_decode: workspace must be 256-byte aligned");
+  (void)workspace;
+  (void)workspace_bytes;
   fa::DecodeParams p;
   p.q = static_cast<const uint16_t*>(q);
   p.k_cache = static_cast<uint16_t*>(k_cache);
@@ -411,26 +398,23 @@ fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cach
   p.nsplit = ns;
   p.chunk = chunk;
   p.scale_log2 = scale * 1.4426950408889634f;
-  if (ns > 1) {
-    const size_t o_bytes = static_cast<size_t>(B) * H * ns * d * sizeof(float);
-    p.part_o = static_cast<float*>(workspace);
-    p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) + (o_bytes + 255) / 256 * 256);
-  } else {
-    p.part_o = nullptr;
-    p.part_lse = nullptr;
-  }
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const dim3 grid(ns, H, B);
-  if (d == 64) fa::decode_split_kernel<64><<<grid, 128, 0, s>>>(p);
-  else fa::decode_split_kernel<128><<<grid, 128, 0, s>>>(p);
-  if ((st = check_launch("fa_decode split kernel launch")) != FA_OK) return st;
-  if (ns > 1) {
-    const unsigned heads = static_cast<unsigned>(B) * H;
-    if (d == 64) fa::decode_merge_kernel<64><<<heads, 64, 0, s>>>(p);
-    else fa::decode_merge_kernel<128><<<heads, 128, 0, s>>>(p);
-    if ((st = check_launch("fa_decode merge kernel launch")) != FA_OK) return st;
-  }
-  return FA_OK;
+  // The `ns` CTAs of one (batch, head) run as one thread-block cluster.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ns, H, B);
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = static_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ns;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = (d == 64) ? cudaLaunchKernelEx(&cfg, fa::decode_kernel<64>, p)
+                            : cudaLaunchKernelEx(&cfg, fa::decode_kernel<128>, p);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_decode kernel launch");
+  return check_launch("fa_decode kernel launch");
 }
 
 fa_status fa_device_status(void* stream, unsigned int* site_out, unsigned int* info_out) {
