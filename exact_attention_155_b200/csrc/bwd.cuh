@@ -159,6 +159,9 @@ struct BwdLayout {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
+// Of every 16 exponential pairs, this many use the FMA-pipe polynomial.
+constexpr int kPolyPairsBwd = 6;
+
 enum : unsigned int {
   kSiteBwdProducer = 0x201,
   kSiteBwdMma = 0x202,
@@ -338,8 +341,9 @@ __global__ void __launch_bounds__(320, 1)
           issue_st(0);
         }
       }
-      // Issue order per query tile n: dV(n), dP^T(n), [S^T(n+1)], dK(n), dQ(n): the
-      // exponentials of tile n+1 overlap the dK/dQ products of tile n.
+      // Issue order per query tile n: dV(n), dP^T(n), S^T(n+1), dK(n), dQ(n): the dS
+      // pass of tile n overlaps S^T(n+1), and the exponentials of tile n+1 overlap the
+      // dK/dQ products of tile n.
       for (int n = 0; n < niter && ok; ++n) {
         const int s = n % L::kQStages;
         const uint32_t sQ = q_addr(n);
@@ -364,9 +368,8 @@ __global__ void __launch_bounds__(320, 1)
         }
         umma_commit(BAR(L::kDPFull));
         umma_commit(BAR(L::kDOEmpty));
-        if (!(ok = wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma))) break;
-        tc_fence_after();
-        // S^T(n+1): the S columns are free (P(n) was read by dV(n); the dS pass is done).
+        // S^T(n+1): the S columns are free once dV(n) (issued above, executed in order)
+        // has read P(n); the dS pass keeps P(n) in registers. It overlaps dS(n).
         if (n + 1 < niter) {
           if (!(ok = wait_bar(BAR(L::kQFull + (n + 1) % L::kQStages), ((n + 1) / L::kQStages) & 1,
                               abort_flag, kSiteBwdMma)))
@@ -374,6 +377,8 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
           issue_st(n + 1);
         }
+        if (!(ok = wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        tc_fence_after();
         // dK += dS^T Q_n
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
@@ -433,8 +438,15 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t* src = c < 32 ? s0 : (c < 64 ? s1 : (c < 96 ? s2 : s3));
         const float x0 = __uint_as_float(src[c & 31]) * sl2 - vec[c];
         const float x1 = __uint_as_float(src[(c + 1) & 31]) * sl2 - vec[c + 1];
-        const float p0 = (c < qlim) ? 0.f : ex2_approx(x0);
-        const float p1 = (c + 1 < qlim) ? 0.f : ex2_approx(x1);
+        float e0 = x0, e1 = x1;
+        if ((c2 & 15) < kPolyPairsBwd) {
+          exp2_poly2(e0, e1);  // FMA/ALU pipes
+        } else {
+          e0 = ex2_approx(e0);  // MUFU
+          e1 = ex2_approx(e1);
+        }
+        const float p0 = (c < qlim) ? 0.f : e0;
+        const float p1 = (c + 1 < qlim) ? 0.f : e1;
         pk[c2] = pack_bf16x2(p0, p1);
       }
       {

@@ -73,7 +73,7 @@ __device__ __forceinline__ void online_merge(float& m, float& l, float (&o)[8], 
 // memory (distributed shared memory), so the whole step is a single launch with no
 // global workspace.
 template <int D>
-__global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(128, 8) decode_kernel(const DecodeParams p) {
   constexpr int LPR = D / 8;     // lanes per cache row (16 bytes each)
   constexpr int RPW = 32 / LPR;  // rows per warp per step
   constexpr int U = 4;           // steps whose loads are issued together
