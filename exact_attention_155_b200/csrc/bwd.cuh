@@ -20,9 +20,11 @@
 //       dK  += dS^T Q_i       (A = dS^T in shared memory, TMEM [256+d,256+2d))
 //       dQ_i = dS K           (A = the same shared buffer read MN-major,
 //                              TMEM cols [128,128+d) once dP^T has been read)
-//    Warps 0-3 (one key row per thread) turn S^T into P^T and dP^T into dS^T;
-//    warps 4-7 (one query row per thread) drain dQ_i from TMEM into the fp32
-//    accumulator with vector atomics; warp 8 issues TMA; warp 9 issues tcgen05.mma.
+//    Warps 0-7 (one key row per thread, two warpgroups splitting the query
+//    columns) turn S^T into P^T and dP^T into dS^T; warps 8-11 drain dQ_i from TMEM
+//    into the fp32 accumulator (shared-memory staging + bulk async reductions for
+//    d = 128, vector atomics for d = 64); warp 12 issues TMA; warp 13 issues
+//    tcgen05.mma.
 //  * bwd_dq_convert_kernel: dq = bf16(accumulator).
 #pragma once
 
@@ -154,13 +156,17 @@ struct BwdLayout {
   static constexpr int kNumBars = kDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = 448;
   static constexpr uint32_t kTmemCols = 512;
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-// Of every 16 exponential pairs, this many use the FMA-pipe polynomial.
-constexpr int kPolyPairsBwd = 6;
+// Of every 16 exponential pairs of the P pass, this many use the FMA-pipe polynomial
+// (exp2_poly2) instead of the MUFU unit.
+#ifndef FA_BWD_POLY_PAIRS
+#define FA_BWD_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairsBwd = FA_BWD_POLY_PAIRS;
 
 enum : unsigned int {
   kSiteBwdProducer = 0x201,
@@ -215,8 +221,11 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                : "memory");
 }
 
+// Trace slot of (role, iteration, event) for the traced CTA (block 0).
+#define FA_BWD_TR(role, n, e) ((((role) * 128 + ((n) & 127)) * 8) + (e))
+
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(448, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                const BwdParams p) {
@@ -252,8 +261,8 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(BAR(L::kDOEmpty), 1);
     mbar_init(BAR(L::kSFull), 1);
     mbar_init(BAR(L::kDPFull), 1);
-    mbar_init(BAR(L::kPFull), 128);
-    mbar_init(BAR(L::kDSFull), 128);
+    mbar_init(BAR(L::kPFull), 256);
+    mbar_init(BAR(L::kDSFull), 256);
     mbar_init(BAR(L::kDSFree), 1);
     mbar_init(BAR(L::kDQFull), 1);
     mbar_init(BAR(L::kDQFree), 128);
@@ -273,7 +282,7 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 128, tDV = tmem + 256,
                  tDK = tmem + 256 + D;
 
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -293,6 +302,7 @@ __global__ void __launch_bounds__(320, 1)
         const int s = n % L::kQStages;
         if (!wait_bar(BAR(L::kQEmpty + s), ((n / L::kQStages) & 1) ^ 1u, abort_flag, kSiteBwdProducer))
           break;
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(3, n, 0));
         const uint32_t sQ = base + L::kQ0 + s * L::kTile;
         mbar_arrive_expect_tx(BAR(L::kQFull + s), L::kTile + 1024);
         for (int bx = 0; bx < D / 64; ++bx)
@@ -302,6 +312,7 @@ __global__ void __launch_bounds__(320, 1)
         bulk_load(sv + 512, dvec_h + it * 128, 512, BAR(L::kQFull + s));
         ++nq;
         if (!wait_bar(BAR(L::kDOEmpty), (n & 1) ^ 1u, abort_flag, kSiteBwdProducer)) break;
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(3, n, 1));
         mbar_arrive_expect_tx(BAR(L::kDOFull), L::kTile);
         for (int bx = 0; bx < D / 64; ++bx)
           tma_load_4d(base + L::kDO + bx * 16384, &tmdO, BAR(L::kDOFull), bx * 64, h, it * 128, b);
@@ -313,7 +324,7 @@ __global__ void __launch_bounds__(320, 1)
       if (ndo > 0) drain_wait(BAR(L::kDOFull), (ndo - 1) & 1);
       drain_wait(BAR(L::kKVFull), 0);
     }
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------- MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
@@ -341,25 +352,21 @@ __global__ void __launch_bounds__(320, 1)
           issue_st(0);
         }
       }
-      // Issue order per query tile n: dV(n), dP^T(n), S^T(n+1), dK(n), dQ(n): the dS
-      // pass of tile n overlaps S^T(n+1), and the exponentials of tile n+1 overlap the
-      // dK/dQ products of tile n.
+      // Issue order per query tile n: dP^T(n), dV(n), S^T(n+1), dQ(n), dK(n): dP^T(n)
+      // overlaps the exponentials of tile n, the dS pass of tile n overlaps dV(n) and
+      // S^T(n+1), the exponentials of tile n+1 overlap dQ(n) and dK(n), and the dQ
+      // drain overlaps dK(n).
       for (int n = 0; n < niter && ok; ++n) {
         const int s = n % L::kQStages;
         const uint32_t sQ = q_addr(n);
-        // dV += P^T dO_n
-        if (!(ok = wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma))) break;
-        if (!(ok = wait_bar(BAR(L::kDOFull), n & 1, abort_flag, kSiteBwdMma))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
-                  (n > 0 || kk > 0) ? 1u : 0u);
-        // dP^T = V dO_n^T, into the columns dQ(n-1) used once they were read out.
+        // dP^T(n) = V dO_n^T, into the columns dQ(n-1) used once they were read out. It
+        // does not need P(n), so the dS pass can start as soon as P(n) is done.
         if (n > 0) {
           if (!(ok = wait_bar(BAR(L::kDQFree), (n - 1) & 1, abort_flag, kSiteBwdMma))) break;
-          tc_fence_after();
         }
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 0));
+        if (!(ok = wait_bar(BAR(L::kDOFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
@@ -367,9 +374,19 @@ __global__ void __launch_bounds__(320, 1)
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(BAR(L::kDPFull));
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 1));
+        // dV += P^T dO_n
+        if (!(ok = wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 2));
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
+                  (n > 0 || kk > 0) ? 1u : 0u);
         umma_commit(BAR(L::kDOEmpty));
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 3));
         // S^T(n+1): the S columns are free once dV(n) (issued above, executed in order)
-        // has read P(n); the dS pass keeps P(n) in registers. It overlaps dS(n).
+        // has read P(n); the dS pass keeps P(n) in registers.
         if (n + 1 < niter) {
           if (!(ok = wait_bar(BAR(L::kQFull + (n + 1) % L::kQStages), ((n + 1) / L::kQStages) & 1,
                               abort_flag, kSiteBwdMma)))
@@ -377,14 +394,11 @@ __global__ void __launch_bounds__(320, 1)
           tc_fence_after();
           issue_st(n + 1);
         }
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 4));
         if (!(ok = wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma))) break;
         tc_fence_after();
-        // dK += dS^T Q_n
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tDK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
-                  sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdKV, (n > 0 || kk > 0) ? 1u : 0u);
-        // dQ_n
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 5));
+        // dQ_n first, so the drain reads it out of TMEM while dK(n) runs.
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           if constexpr (D == 128)
@@ -395,50 +409,58 @@ __global__ void __launch_bounds__(320, 1)
                     sdesc_sw128(sK + kk * 2048, 16384, 1024), kIdQ, kk > 0 ? 1u : 0u);
         }
         umma_commit(BAR(L::kDQFull));
+        // dK += dS^T Q_n
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tDK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+                  sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdKV, (n > 0 || kk > 0) ? 1u : 0u);
         umma_commit(BAR(L::kDSFree));
         umma_commit(BAR(L::kQEmpty + s));
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 6));
       }
       if (ok) umma_commit(BAR(L::kMmaDone));
       umma_commit(BAR(L::kDrain));
       drain_wait(BAR(L::kDrain), 0);
     }
-  } else if (warp < 4) {
-    // -------------------------------------------- P^T and dS^T (one key per thread)
-    const int r = warp * 32 + lane;
+  } else if (warp < 8) {
+    // ------------------------------------ P^T and dS^T: one key row per thread; two
+    // warpgroups split the 128 query columns of every tile (64 columns each).
+    const int wq = warp & 3;
+    const int half = warp >> 2;
+    const int c0 = half * 64;  // first query column of this warpgroup
+    const int r = wq * 32 + lane;
     const int key = jt * 128 + r;
     const bool key_ok = key < p.N;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float sl2 = p.scale_log2;
+    const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
     bool ok = true;
     for (int n = 0; n < niter; ++n) {
       const int it = it0 + n;
       const int s = n % L::kQStages;
-      const float* vec = reinterpret_cast<const float*>(smem + L::kVec + s * 1024);
+      const float* vec = reinterpret_cast<const float*>(smem + L::kVec + s * 1024) + c0;
       ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kSFull), n & 1, abort_flag, kSiteBwdSoftmax));
       if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kQFull + s), (n / L::kQStages) & 1,
                                                    abort_flag, kSiteBwdSoftmax));
       if (!ok) break;
+      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 0));
       tc_fence_after();
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(tS + lane_off + 0, s0);
-      tmem_ld32(tS + lane_off + 32, s1);
-      tmem_ld32(tS + lane_off + 64, s2);
-      tmem_ld32(tS + lane_off + 96, s3);
+      uint32_t s0[32], s1[32];
+      tmem_ld32(tS + lane_off + c0, s0);
+      tmem_ld32(tS + lane_off + c0 + 32, s1);
       tmem_wait_ld();
       reg_fence32(s0);
       reg_fence32(s1);
-      reg_fence32(s2);
-      reg_fence32(s3);
-      // Queries of this tile that key `key` may not attend: q < key (causal) or key >= N.
-      const int qlim = !key_ok ? 1 << 30 : (CAUSAL ? key - it * 128 : 0);
-      uint32_t pk[64];
+      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 1));
+      // Local columns c < qlim are not visible to this key: query < key (causal) or key >= N.
+      const int qlim = !key_ok ? 1 << 30 : (CAUSAL ? key - it * 128 - c0 : 0);
+      uint32_t pk[32];
 #pragma unroll
-      for (int c2 = 0; c2 < 64; ++c2) {
+      for (int c2 = 0; c2 < 32; ++c2) {
         const int c = 2 * c2;
-        const uint32_t* src = c < 32 ? s0 : (c < 64 ? s1 : (c < 96 ? s2 : s3));
-        const float x0 = __uint_as_float(src[c & 31]) * sl2 - vec[c];
-        const float x1 = __uint_as_float(src[(c + 1) & 31]) * sl2 - vec[c + 1];
-        float e0 = x0, e1 = x1;
+        const uint32_t* src = c < 32 ? s0 : s1;
+        float e0 = __uint_as_float(src[c & 31]) * sl2 - vec[c];
+        float e1 = __uint_as_float(src[(c + 1) & 31]) * sl2 - vec[c + 1];
         if ((c2 & 15) < kPolyPairsBwd) {
           exp2_poly2(e0, e1);  // FMA/ALU pipes
         } else {
@@ -449,32 +471,28 @@ __global__ void __launch_bounds__(320, 1)
         const float p1 = (c + 1 < qlim) ? 0.f : e1;
         pk[c2] = pack_bf16x2(p0, p1);
       }
-      {
-        uint32_t a[32], bq[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          a[c] = pk[c];
-          bq[c] = pk[32 + c];
-        }
-        tmem_st32(tS + lane_off + 0, a);
-        tmem_st32(tS + lane_off + 32, bq);
-      }
+      tmem_st32(tS + lane_off + c0 / 2, pk);  // P^T bf16: two queries per 32-bit column
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(L::kPFull));
+      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 2));
 
       ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDPFull), n & 1, abort_flag, kSiteBwdSoftmax));
       if (ok && n > 0)
         ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDSFree), (n - 1) & 1, abort_flag, kSiteBwdSoftmax));
       if (!ok) break;
+      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 3));
       tc_fence_after();
       const float* dvec = vec + 128;
+      uint32_t dp0[32], dp1[32];
+      tmem_ld32(tDP + lane_off + c0, dp0);
+      tmem_ld32(tDP + lane_off + c0 + 32, dp1);
+      tmem_wait_ld();
+      reg_fence32(dp0);
+      reg_fence32(dp1);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t dp[32];
-        tmem_ld32(tDP + lane_off + q * 32, dp);
-        tmem_wait_ld();
-        reg_fence32(dp);
+      for (int q = 0; q < 2; ++q) {
+        const uint32_t* dp = q == 0 ? dp0 : dp1;
         uint32_t w[16];
 #pragma unroll
         for (int c2 = 0; c2 < 16; ++c2) {
@@ -485,11 +503,11 @@ __global__ void __launch_bounds__(320, 1)
           const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1]) - dvec[c + 1]);
           w[c2] = pack_bf16x2(d0, d1);
         }
-        // Row r of the dS^T tile, queries q*32 .. q*32+31, 128-byte swizzle.
-        const uint32_t row_base = sDS + (q >> 1) * 16384 + r * 128;
+        // Row r of the dS^T tile, queries c0 + q*32 .. +31 (box `half`), 128-byte swizzle.
+        const uint32_t row_base = sDS + half * 16384 + r * 128;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = (q & 1) * 4 + ch;
+          const int chunk = q * 4 + ch;
           st_shared_v4(row_base + ((chunk ^ (r & 7)) << 4), w[4 * ch], w[4 * ch + 1], w[4 * ch + 2],
                        w[4 * ch + 3]);
         }
@@ -497,35 +515,34 @@ __global__ void __launch_bounds__(320, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(BAR(L::kDSFull));
+      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 4));
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kMmaDone), 0, abort_flag, kSiteBwdSoftmax));
     if (ok) {
+      // Epilogue: warpgroup 0 writes dV rows, warpgroup 1 writes dK rows (x scale).
       tc_fence_after();
       const size_t orow = ((static_cast<size_t>(b) * p.N + key) * p.H + h) * D;
+      const uint32_t tsrc = (half == 0 ? tDV : tDK) + lane_off;
+      const float mul = half == 0 ? 1.f : p.scale;
+      uint16_t* dst = (half == 0 ? p.dv : p.dk) + orow;
 #pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tsrc = (which == 0 ? tDV : tDK) + lane_off;
-        const float mul = which == 0 ? 1.f : p.scale;
-        uint16_t* dst = (which == 0 ? p.dv : p.dk) + orow;
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tsrc + cc * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
+        if (key_ok) {
+          uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
 #pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tsrc + cc * 32, o);
-          tmem_wait_ld();
-          reg_fence32(o);
-          if (key_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v)
-              d4[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * mul, __uint_as_float(o[8 * v + 1]) * mul),
-                                 pack_bf16x2(__uint_as_float(o[8 * v + 2]) * mul, __uint_as_float(o[8 * v + 3]) * mul),
-                                 pack_bf16x2(__uint_as_float(o[8 * v + 4]) * mul, __uint_as_float(o[8 * v + 5]) * mul),
-                                 pack_bf16x2(__uint_as_float(o[8 * v + 6]) * mul, __uint_as_float(o[8 * v + 7]) * mul));
-          }
+          for (int v = 0; v < 4; ++v)
+            d4[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * mul, __uint_as_float(o[8 * v + 1]) * mul),
+                               pack_bf16x2(__uint_as_float(o[8 * v + 2]) * mul, __uint_as_float(o[8 * v + 3]) * mul),
+                               pack_bf16x2(__uint_as_float(o[8 * v + 4]) * mul, __uint_as_float(o[8 * v + 5]) * mul),
+                               pack_bf16x2(__uint_as_float(o[8 * v + 6]) * mul, __uint_as_float(o[8 * v + 7]) * mul));
         }
       }
     }
-  } else {
+  } else if (warp < 12) {
     // ------------------------------------------------------------- dQ drain
     // d = 128: TMEM holds dQ^T (lane = head-dim index j, column = query), so one warp
     // instruction reduces 32 consecutive floats of one dQ row (128 contiguous bytes).
@@ -540,6 +557,7 @@ __global__ void __launch_bounds__(320, 1)
       // All four drain warps leave together: they share named barriers below.
       ok = named_bar_and(1, 128, ok);
       if (!ok) break;
+      FA_TRACE_EVENT(blockIdx.x == 0 && threadIdx.x == 256, FA_BWD_TR(2, n, 0));
       tc_fence_after();
       if constexpr (D == 128) {
         // Read all of dQ^T (128 queries for this thread's head-dim index r), free the
@@ -558,8 +576,9 @@ __global__ void __launch_bounds__(320, 1)
         reg_fence32(o3);
         tc_fence_before();
         mbar_arrive(BAR(L::kDQFree));
+        FA_TRACE_EVENT(blockIdx.x == 0 && threadIdx.x == 256, FA_BWD_TR(2, n, 1));
         float* gtile = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(it) * 128) * D;
-        const bool leader = (warp == 4 && lane == 0);
+        const bool leader = (warp == 8 && lane == 0);
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc) {
           const uint32_t buf = base + L::kStage + (cc & 1) * 16384;
@@ -575,6 +594,7 @@ __global__ void __launch_bounds__(320, 1)
             bulk_commit();
           }
         }
+        FA_TRACE_EVENT(blockIdx.x == 0 && threadIdx.x == 256, FA_BWD_TR(2, n, 2));
         continue;
       } else {
         const int qrow = it * 128 + r;
@@ -598,7 +618,7 @@ __global__ void __launch_bounds__(320, 1)
       mbar_arrive(BAR(L::kDQFree));
     }
     if constexpr (D == 128) {
-      if (warp == 4 && lane == 0) bulk_wait_all();  // reductions complete before exit
+      if (warp == 8 && lane == 0) bulk_wait_all();  // reductions complete before exit
     }
   }
 

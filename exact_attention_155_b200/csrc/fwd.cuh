@@ -61,10 +61,6 @@ struct FwdLayout {
   static constexpr uint32_t kTmemCols = 512;
 };
 
-// Of every 16 exponential pairs in an unmasked tile, this many go to the FMA-pipe
-// polynomial (exp2_poly2) and the rest to the MUFU unit.
-constexpr int kPolyPairs = 6;
-
 // Site ids for timeout reports.
 enum : unsigned int { kSiteFwdProducer = 0x101, kSiteFwdMma = 0x102, kSiteFwdSoftmax = 0x103 };
 
@@ -329,17 +325,13 @@ __global__ void __launch_bounds__(320, 1)
           const int c = ch * 32 + 2 * i;
           float a = x[c], bb = x[c + 1];
           if (masked) {
-            a = ex2_approx(a - ms);
-            bb = ex2_approx(bb - ms);
+            a -= ms;
+            bb -= ms;
           } else {
             fma2(a, bb, a, bb, sl2, sl2, nms, nms);
-            if (i < kPolyPairs) {
-              exp2_poly2(a, bb);  // FMA/ALU pipes
-            } else {
-              a = ex2_approx(a);  // MUFU
-              bb = ex2_approx(bb);
-            }
           }
+          a = ex2_approx(a);
+          bb = ex2_approx(bb);
           add2(rs0, rs1, rs0, rs1, a, bb);
           pk[i] = pack_bf16x2(a, bb);
         }
