@@ -64,6 +64,9 @@ struct FwdLayout {
 // Site ids for timeout reports.
 enum : unsigned int { kSiteFwdProducer = 0x101, kSiteFwdMma = 0x102, kSiteFwdSoftmax = 0x103 };
 
+// Trace slot of (role, key tile, event) for the traced CTA (block 0).
+#define FA_FWD_TR(role, j, e) ((((role) * 128 + ((j) & 127)) * 8) + (e))
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(320, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -145,6 +148,7 @@ __global__ void __launch_bounds__(320, 1)
             stop = true;
             break;
           }
+          FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(3, j, kv));
           mbar_arrive_expect_tx(BAR(L::kKVFull + s), L::kTileBytes);
           const CUtensorMap* m = kv ? &tmV : &tmK;
           for (int bx = 0; bx < D / 64; ++bx)
@@ -207,6 +211,7 @@ __global__ void __launch_bounds__(320, 1)
           ok = false;
           break;
         }
+        FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(0, j, 0));
         tc_fence_after();
         bool k_next = false;
         for (int t = 0; t < 2; ++t) {
@@ -215,6 +220,7 @@ __global__ void __launch_bounds__(320, 1)
             ok = false;
             break;
           }
+          FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(0, j, 1 + 2 * t));
           tc_fence_after();
           issue_pv(t, sv, j > 0);
           if (j + 1 < nkv[t]) {
@@ -232,6 +238,7 @@ __global__ void __launch_bounds__(320, 1)
           } else {
             umma_commit(BAR(L::kOFinal + t));
           }
+          FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(0, j, 2 + 2 * t));
         }
         if (!ok) break;
         umma_commit(BAR(L::kKVEmpty + sv));
@@ -259,6 +266,7 @@ __global__ void __launch_bounds__(320, 1)
       ok = __all_sync(0xffffffffu,
                       wait_bar(BAR(L::kSFull + t), j & 1, abort_flag, kSiteFwdSoftmax));
       if (!ok) break;
+      FA_TRACE_EVENT(blockIdx.x == 0 && (threadIdx.x & 127) == 0, FA_FWD_TR(1 + t, j, 0));
       tc_fence_after();
       uint32_t s0[32], s1[32], s2[32], s3[32];
       tmem_ld32(tS + 0, s0);
@@ -270,6 +278,7 @@ __global__ void __launch_bounds__(320, 1)
       reg_fence32(s1);
       reg_fence32(s2);
       reg_fence32(s3);
+      FA_TRACE_EVENT(blockIdx.x == 0 && (threadIdx.x & 127) == 0, FA_FWD_TR(1 + t, j, 1));
       float x[128];
 #pragma unroll
       for (int c = 0; c < 32; ++c) {
@@ -360,6 +369,7 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(L::kPFull + t));
+      FA_TRACE_EVENT(blockIdx.x == 0 && (threadIdx.x & 127) == 0, FA_FWD_TR(1 + t, j, 2));
     }
     if (ok && nkv[t] > 0) {
       ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kOFinal + t), 0, abort_flag, kSiteFwdSoftmax));
