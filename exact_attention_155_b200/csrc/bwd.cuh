@@ -37,6 +37,7 @@ namespace fa {
 struct BwdParams {
   int B, H, N, Np;      // Np = N rounded up to a multiple of 128
   int nqt;              // Np / 128
+  int head_group;       // heads scheduled together (divides B*H), for L2 reuse
   float scale;          // softmax scale
   float scale_log2;     // scale * log2(e)
   const uint16_t* out;  // forward output [B, N, H, d]
@@ -197,22 +198,6 @@ __device__ __forceinline__ void bulk_wait_read1() {
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
-// Barrier over `nthreads` threads that also returns the AND of every thread's predicate.
-__device__ __forceinline__ bool named_bar_and(int id, int nthreads, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred pi, po;\n\t"
-      "setp.ne.u32 pi, %1, 0;\n\t"
-      "bar.red.and.pred po, %2, %3, pi;\n\t"
-      "selp.u32 %0, 1, 0, po;\n\t}"
-      : "=r"(r)
-      : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
 __device__ __forceinline__ void st_shared_f32(uint32_t addr, float v) {
   asm volatile("st.shared.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
@@ -245,8 +230,14 @@ __global__ void __launch_bounds__(448, 1)
 
   const int warp = warp_id(), lane = lane_id();
   const int BH = p.B * p.H;
-  const int jt = static_cast<int>(blockIdx.x) / BH;  // key tile; low ids = most work when causal
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  // Heads in groups of head_group (L2 reuse of Q/dO and the dQ accumulator); within a
+  // group, key tile 0 (the most query tiles when causal) first.
+  const int G = p.head_group;
+  const int per_group = G * p.nqt;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int rem = static_cast<int>(blockIdx.x) % per_group;
+  const int jt = rem / G;
+  const int bh = grp * G + rem % G;
   const int b = bh / p.H, h = bh % p.H;
   const int it0 = CAUSAL ? jt : 0;
   const int niter = p.nqt - it0;

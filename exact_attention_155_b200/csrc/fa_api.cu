@@ -38,6 +38,14 @@ fa_status cuda_fail(cudaError_t e, const char* what) {
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Largest divisor of n that is <= cap: the number of heads whose CTAs are scheduled
+// together so their K/V (or Q/dO) stay resident in L2.
+int head_group_for(int n, int cap) {
+  for (int g = cap < n ? cap : n; g > 1; --g)
+    if (n % g == 0) return g;
+  return 1;
+}
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 // ---------------------------------------------------------------- device info
@@ -198,6 +206,8 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   p.N = N;
   p.Np = (N + 127) / 128 * 128;
   p.nqt = p.Np / 128;
+  // Four heads: their Q, dO and fp32 dQ accumulator (4 x 16 MiB at N = 16384) fit in L2.
+  p.head_group = head_group_for(B * H, 4);
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = static_cast<const uint16_t*>(out);
@@ -306,6 +316,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   p.H = H;
   p.N = N;
   p.num_qblocks = static_cast<int>(nqb);
+  // Eight heads: their K and V (8 x 4 MiB at N = 8192) stay in L2 while their CTAs run.
+  p.head_group = head_group_for(B * H, 8);
   p.nkv_total = (N + 127) / 128;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.out = static_cast<uint16_t*>(out);

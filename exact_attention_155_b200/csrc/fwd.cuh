@@ -16,10 +16,12 @@
 //  * warp 9 issues tcgen05.mma from one thread: S_t = Q_t K_j^T into TMEM
 //    (fp32, 128 lanes x 128 columns per tile), then O_t += P_t V_j with P_t read
 //    straight from TMEM (bf16 packed over the first 64 columns of S_t);
-//  * warps 0-3 and 4-7 are the softmax warpgroups of tiles 0 and 1; each thread
-//    owns one query row (one TMEM lane), so row max and row sum need no shuffles.
-//    The two groups alternate with the tensor core: while one does exp, the MMA
-//    warp computes the other tile's products;
+//  * warps 0-7 do the softmax of one Q tile at a time (tile 0, then tile 1, per key
+//    tile): warps 0-3 take key columns 0-63 and warps 4-7 columns 64-127 of the
+//    same 128 rows (one TMEM lane per row), so all eight warps keep the exponential
+//    unit busy while the MMA warp computes the other tile's products; both halves
+//    read the whole row of scores for the row max, and each half publishes its P
+//    columns to the MMA warp as soon as they are stored;
 //  * TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+d) O_1 [256+d,256+2d).
 #pragma once
 
@@ -32,6 +34,7 @@ namespace fa {
 struct FwdParams {
   int B, H, N;
   int num_qblocks;   // ceil(N / 256): CTAs per (batch, head)
+  int head_group;    // heads scheduled together (divides B*H), for L2 reuse of K/V
   int nkv_total;     // ceil(N / 128): key tiles per head
   float scale_log2;  // scale * log2(e)
   uint16_t* out;     // [B, N, H, d] bf16
@@ -50,19 +53,53 @@ struct FwdLayout {
   static constexpr int kKVFull = 2;                     // [kStages]
   static constexpr int kKVEmpty = 2 + kStages;          // [kStages]
   static constexpr int kSFull = 2 + 2 * kStages;        // [2]
-  static constexpr int kPFull = kSFull + 2;             // [2]
-  static constexpr int kOFinal = kPFull + 2;            // [2]
+  static constexpr int kPHalf = kSFull + 2;             // [2 tiles][2 key halves]
+  static constexpr int kOFinal = kPHalf + 4;            // [2]
   static constexpr int kDrain = kOFinal + 2;            // [1]
   static constexpr int kNumBars = kDrain + 1;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  // Exchange between the two column halves of a row: maxima [tile][half][128] fp32
+  // (exact steps only) and exp-sums [tile][half][128] fp32 (epilogue).
+  static constexpr int kXMaxOff = kBarOff + kNumBars * 8;
+  static constexpr int kXSumOff = kXMaxOff + 2 * 2 * 128 * 4;
+  static constexpr int kMiscOff = kXSumOff + 2 * 2 * 128 * 4;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kThreads = 320;
   static constexpr uint32_t kTmemCols = 512;
 };
 
+// Of every 16 exponential pairs of an unmasked tile, this many use the FMA-pipe
+// polynomial (exp2_poly2) instead of the MUFU unit.
+#ifndef FA_FWD_POLY_PAIRS
+#define FA_FWD_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
+
 // Site ids for timeout reports.
 enum : unsigned int { kSiteFwdProducer = 0x101, kSiteFwdMma = 0x102, kSiteFwdSoftmax = 0x103 };
+
+// Max / min of 128 values held as two 64-element halves, with 8 independent
+// accumulators so the reduction is 10 dependent steps deep instead of 64.
+__device__ __forceinline__ float row_max128(const float (&x)[64], const float (&y)[64]) {
+  float acc[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) acc[a] = fmaxf(x[a], y[a]);
+#pragma unroll
+  for (int c = 8; c < 64; c += 8)
+#pragma unroll
+    for (int a = 0; a < 8; ++a) acc[a] = max3f(acc[a], x[c + a], y[c + a]);
+  return fmaxf(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], max3f(acc[5], acc[6], acc[7])));
+}
+__device__ __forceinline__ float row_min128(const float (&x)[64], const float (&y)[64]) {
+  float acc[8];
+#pragma unroll
+  for (int a = 0; a < 8; ++a) acc[a] = fminf(x[a], y[a]);
+#pragma unroll
+  for (int c = 8; c < 64; c += 8)
+#pragma unroll
+    for (int a = 0; a < 8; ++a) acc[a] = min3f(acc[a], x[c + a], y[c + a]);
+  return fminf(min3f(acc[0], acc[1], acc[2]), min3f(acc[3], acc[4], min3f(acc[5], acc[6], acc[7])));
+}
 
 // Trace slot of (role, key tile, event) for the traced CTA (block 0).
 #define FA_FWD_TR(role, j, e) ((((role) * 128 + ((j) & 127)) * 8) + (e))
@@ -86,10 +123,14 @@ __global__ void __launch_bounds__(320, 1)
   const int warp = warp_id();
   const int lane = lane_id();
 
-  // Work unit: heaviest causal row blocks get the lowest block ids.
-  const int BH = p.B * p.H;
-  const int qb = p.num_qblocks - 1 - static_cast<int>(blockIdx.x) / BH;
-  const int bh = static_cast<int>(blockIdx.x) % BH;
+  // Work unit: heads are taken in groups of head_group so the CTAs in flight share
+  // a few heads' K/V in L2; within a group the heaviest causal row blocks come first.
+  const int G = p.head_group;
+  const int per_group = G * p.num_qblocks;
+  const int grp = static_cast<int>(blockIdx.x) / per_group;
+  const int rem = static_cast<int>(blockIdx.x) % per_group;
+  const int qb = p.num_qblocks - 1 - rem / G;
+  const int bh = grp * G + rem % G;
   const int b = bh / p.H;
   const int h = bh % p.H;
   int row0[2], nkv[2];
@@ -105,7 +146,8 @@ __global__ void __launch_bounds__(320, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(BAR(L::kQFull + t), 1);
       mbar_init(BAR(L::kSFull + t), 1);
-      mbar_init(BAR(L::kPFull + t), 128);
+      mbar_init(BAR(L::kPHalf + 2 * t + 0), 128);
+      mbar_init(BAR(L::kPHalf + 2 * t + 1), 128);
       mbar_init(BAR(L::kOFinal + t), 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
@@ -180,11 +222,13 @@ __global__ void __launch_bounds__(320, 1)
           umma_ss(dt, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
         }
       };
-      auto issue_pv = [&](int t, int s, bool acc) {
+      // O_t += P_t V for keys [64*half, 64*half + 64) of the tile.
+      auto issue_pv_half = [&](int t, int s, int half, bool acc) {
         const uint32_t dt = tmem + 256 + t * D;
         const uint32_t at = tmem + t * 128;
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = half * 4 + k4;
           const uint64_t bd = sdesc_sw128(sKV + s * L::kTileBytes + kk * 2048, 16384, 1024);
           umma_ts(dt, at + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
         }
@@ -216,13 +260,21 @@ __global__ void __launch_bounds__(320, 1)
         bool k_next = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= nkv[t]) continue;
-          if (!wait_bar(BAR(L::kPFull + t), j & 1, abort_flag, kSiteFwdMma)) {
+          // P_t arrives in two key halves; the first half's products start while the
+          // softmax warpgroup is still exponentiating the second half.
+          if (!wait_bar(BAR(L::kPHalf + 2 * t + 0), j & 1, abort_flag, kSiteFwdMma)) {
             ok = false;
             break;
           }
           FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(0, j, 1 + 2 * t));
           tc_fence_after();
-          issue_pv(t, sv, j > 0);
+          issue_pv_half(t, sv, 0, j > 0);
+          if (!wait_bar(BAR(L::kPHalf + 2 * t + 1), j & 1, abort_flag, kSiteFwdMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv_half(t, sv, 1, j > 0);
           if (j + 1 < nkv[t]) {
             if (!k_next) {
               if (!wait_bar(BAR(L::kKVFull + sk), (ik / L::kStages) & 1, abort_flag,
@@ -249,157 +301,214 @@ __global__ void __launch_bounds__(320, 1)
       drain_wait(BAR(L::kDrain), 0);
     }
   } else {
-    // ------------------------------------------------------- softmax warpgroups
-    const int t = warp >> 2;
+    // ------------------------------------------------------------ softmax warps
+    // All eight warps work on one Q tile at a time (tile 0, then tile 1, for every
+    // key tile j): warpgroup `half` takes key columns [64*half, 64*half + 64) of each
+    // of the 128 rows, so the exponential unit is shared by two warps per SM
+    // sub-partition while the MMA warp runs the other tile's products. The two
+    // halves of a row both read the whole row of scores for the row max, and add
+    // their exp-sums through shared memory at the end; P is published to the MMA
+    // warp per half.
+    const int half = warp >> 2;
     const int wq = warp & 3;
     const int r = wq * 32 + lane;
-    const int row_g = row0[t] + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tS = tmem + t * 128 + lane_off;
-    const uint32_t tO = tmem + 256 + t * D + lane_off;
-    const int diag_j = CAUSAL ? row0[t] / 128 : -1;
     const float sl2 = p.scale_log2;
-    float m = -INFINITY;  // running max, log2-scaled units
-    float l = 0.f;        // running exp-sum
+    float* xmax = reinterpret_cast<float*>(smem + L::kXMaxOff);
+    float* xsum = reinterpret_cast<float*>(smem + L::kXSumOff);
+    const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
+    float m[2] = {-INFINITY, -INFINITY};  // running row max per tile (log2 units)
+    float l[2] = {0.f, 0.f};              // running exp-sum over this half's columns
     bool ok = true;
-    for (int j = 0; j < nkv[t]; ++j) {
-      ok = __all_sync(0xffffffffu,
-                      wait_bar(BAR(L::kSFull + t), j & 1, abort_flag, kSiteFwdSoftmax));
-      if (!ok) break;
-      FA_TRACE_EVENT(blockIdx.x == 0 && (threadIdx.x & 127) == 0, FA_FWD_TR(1 + t, j, 0));
+    for (int j = 0; j < nkv_max && ok; ++j) {
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (j >= nkv[t]) continue;  // uniform over the CTA
+        const int row_g = row0[t] + r;
+        const uint32_t tS = tmem + t * 128 + lane_off;
+        const uint32_t tO = tmem + 256 + t * D + lane_off;
+        const bool w_ok = __all_sync(0xffffffffu,
+                                     wait_bar(BAR(L::kSFull + t), j & 1, abort_flag, kSiteFwdSoftmax));
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 0));
+        tc_fence_after();
+        uint32_t s0[32], s1[32];
+        tmem_ld32(tS + 64 * half, s0);
+        tmem_ld32(tS + 64 * half + 32, s1);
+        tmem_wait_ld();
+        reg_fence32(s0);
+        reg_fence32(s1);
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 1));
+        float x[64];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          x[c] = __uint_as_float(s0[c]);
+          x[32 + c] = __uint_as_float(s1[c]);
+        }
+        const int kbase = j * 128 + 64 * half;  // key index of column 0 of this half
+        const bool masked = (CAUSAL && j * 128 == row0[t]) || (j * 128 + 128 > p.N);
+        if (masked) {
+          // Diagonal or tail tile: scale first, then mask to -inf.
+          const int lim = CAUSAL ? min(row_g, p.N - 1) : p.N - 1;
+#pragma unroll
+          for (int c = 0; c < 64; ++c) x[c] = (kbase + c > lim) ? -INFINITY : x[c] * sl2;
+        }
+        // x holds raw scores (unmasked tile) or scaled, masked scores (masked tile).
+        // exps(ms, mx_out): p = 2^(x*sl2 - ms) (resp. 2^(x - ms)) for this half's 64
+        // columns, their sum, bf16 P into TMEM, and this half's max of the scaled
+        // scores computed alongside on the ALU (8 independent accumulators).
+        float rsum = 0.f;
+        auto exps = [&](float ms, float& mx_out) {
+          const float nms = -ms;
+          float rs[4] = {0.f, 0.f, 0.f, 0.f};
+          float acc[8];
+#pragma unroll
+          for (int a8 = 0; a8 < 8; ++a8) acc[a8] = -INFINITY;
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int c = ch * 32 + 2 * i;
+              float a = x[c], bb = x[c + 1];
+              acc[i & 7] = max3f(acc[i & 7], a, bb);
+              if (masked) {
+                a -= ms;
+                bb -= ms;
+              } else {
+                fma2(a, bb, a, bb, sl2, sl2, nms, nms);
+              }
+              if (!masked && i < kPolyPairs) {
+                exp2_poly2(a, bb);  // FMA/ALU pipes
+              } else {
+                a = ex2_approx(a);  // MUFU
+                bb = ex2_approx(bb);
+              }
+              add2(rs[2 * (i & 1)], rs[2 * (i & 1) + 1], rs[2 * (i & 1)], rs[2 * (i & 1) + 1], a, bb);
+              pk[i] = pack_bf16x2(a, bb);
+            }
+            tmem_st16(tS + 32 * half + ch * 16, pk);
+          }
+          float mxr = fmaxf(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], max3f(acc[5], acc[6], acc[7])));
+          mx_out = masked ? mxr : mxr * sl2;
+          rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        };
+        // Fast path: exponentiate against the current reference max while computing
+        // this half's max; if no row of the tile grew past the reference by more than
+        // 2^8, P is final (p <= 256 stays exact enough in fp32 and bf16, and O / l stays
+        // exact because both use the same reference).
+        // The fast/exact choice is uniform over all 256 softmax threads (j and the
+        // scale's sign are), so every thread reaches the same named barriers; an
+        // abort is folded into the vote and forces the exact path, which ends it.
+        bool exact = (j == 0) || !(sl2 >= 0.f);
+        float mx_half = -INFINITY;
+        if (!exact) {
+          exps(m[t], mx_half);
+          exact = named_bar_or(1, 256, !w_ok || !(mx_half <= m[t] + 8.f));
+          if (!exact) l[t] += rsum;
+        }
+        if (exact) {
+          // Exact path (first tile, negative scale, a grown row, or an abort): the two
+          // halves exchange their maxima, move the reference, rescale O, and (re)do
+          // the exponentials.
+          if (mx_half == -INFINITY) {
+            float acc[8];
+#pragma unroll
+            for (int a8 = 0; a8 < 8; ++a8) acc[a8] = (sl2 >= 0.f || masked) ? -INFINITY : INFINITY;
+            if (masked || sl2 >= 0.f) {
+#pragma unroll
+              for (int c = 0; c < 64; c += 2) acc[(c >> 1) & 7] = max3f(acc[(c >> 1) & 7], x[c], x[c + 1]);
+              const float mxr = fmaxf(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], max3f(acc[5], acc[6], acc[7])));
+              mx_half = masked ? mxr : mxr * sl2;
+            } else {
+#pragma unroll
+              for (int c = 0; c < 64; c += 2) acc[(c >> 1) & 7] = min3f(acc[(c >> 1) & 7], x[c], x[c + 1]);
+              mx_half = fminf(min3f(acc[0], acc[1], acc[2]), min3f(acc[3], acc[4], min3f(acc[5], acc[6], acc[7]))) * sl2;
+            }
+          }
+          float* xm = xmax + t * 256;
+          xm[half * 128 + r] = mx_half;
+          ok = named_bar_and(1, 256, w_ok);
+          if (!ok) break;
+          const float mx = fmaxf(mx_half, xm[(half ^ 1) * 128 + r]);
+          const float m_new = fmaxf(m[t], mx);
+          if (__any_sync(0xffffffffu, m_new > m[t] + 8.f)) {
+            const float alpha = ex2_approx(m[t] - m_new);  // 0 on the first tile (m = -inf)
+            l[t] *= alpha;
+            m[t] = m_new;
+            if (j > 0) {
+              // Rescale this half of the row's partial output before this tile's
+              // products accumulate into it (PV_t(j-1) completed before S_t(j)).
+#pragma unroll
+              for (int cc = 0; cc < D / 32; ++cc) {
+                uint32_t o[16];
+                tmem_ld16(tO + half * (D / 2) + cc * 16, o);
+                tmem_wait_ld();
+                reg_fence16(o);
+#pragma unroll
+                for (int c = 0; c < 16; c += 2) {
+                  float a0, a1;
+                  mul2(a0, a1, __uint_as_float(o[c]), __uint_as_float(o[c + 1]), alpha, alpha);
+                  o[c] = __float_as_uint(a0);
+                  o[c + 1] = __float_as_uint(a1);
+                }
+                tmem_st16(tO + half * (D / 2) + cc * 16, o);
+              }
+            }
+          }
+          // The exchange slots are reused at the next exact step of this tile only
+          // after every thread has read them.
+          named_bar_sync(1, 256);
+          float unused;
+          exps(m[t] == -INFINITY ? 0.f : m[t], unused);
+          l[t] += rsum;
+        }
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 4));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(BAR(L::kPHalf + 2 * t + half));
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 2));
+      }
+    }
+    // Epilogue per tile: O / l and the LSE. Each half writes its D/2 output columns.
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      if (nkv[t] == 0) continue;  // uniform over the CTA
+      // Every softmax thread reaches the barrier below, aborted or not; the AND
+      // carries the abort so all 256 threads leave together.
+      bool w_ok = ok;
+      if (w_ok) w_ok = wait_bar(BAR(L::kOFinal + t), 0, abort_flag, kSiteFwdSoftmax);
+      w_ok = __all_sync(0xffffffffu, w_ok);
+      float* xs = xsum + t * 256;
+      xs[half * 128 + r] = l[t];
+      ok = named_bar_and(2, 256, w_ok);
+      if (!ok) continue;
+      const float lt = l[t] + xs[(half ^ 1) * 128 + r];
       tc_fence_after();
-      uint32_t s0[32], s1[32], s2[32], s3[32];
-      tmem_ld32(tS + 0, s0);
-      tmem_ld32(tS + 32, s1);
-      tmem_ld32(tS + 64, s2);
-      tmem_ld32(tS + 96, s3);
-      tmem_wait_ld();
-      reg_fence32(s0);
-      reg_fence32(s1);
-      reg_fence32(s2);
-      reg_fence32(s3);
-      FA_TRACE_EVENT(blockIdx.x == 0 && (threadIdx.x & 127) == 0, FA_FWD_TR(1 + t, j, 1));
-      float x[128];
+      const int row_g = row0[t] + r;
+      const uint32_t tO = tmem + 256 + t * D + lane_off + half * (D / 2);
+      const float inv_l = (lt > 0.f) ? 1.f / lt : 0.f;
+      const bool row_ok = row_g < p.N;
+      uint16_t* orow = p.out + ((static_cast<size_t>(b) * p.N + row_g) * p.H + h) * D + half * (D / 2);
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        x[c] = __uint_as_float(s0[c]);
-        x[32 + c] = __uint_as_float(s1[c]);
-        x[64 + c] = __uint_as_float(s2[c]);
-        x[96 + c] = __uint_as_float(s3[c]);
-      }
-      const int kbase = j * 128;
-      const bool masked = (j == diag_j) || (kbase + 128 > p.N);
-      float mx;
-      if (masked) {
-        // Diagonal or tail tile: scale first, then mask to -inf.
-        const int lim = CAUSAL ? min(row_g, p.N - 1) : p.N - 1;
-#pragma unroll
-        for (int c = 0; c < 128; ++c) x[c] = (kbase + c > lim) ? -INFINITY : x[c] * sl2;
-        mx = x[0];
-#pragma unroll
-        for (int c = 1; c < 127; c += 2) mx = max3f(mx, x[c], x[c + 1]);
-        mx = fmaxf(mx, x[127]);
-      } else if (sl2 >= 0.f) {
-        mx = x[0];
-#pragma unroll
-        for (int c = 1; c < 127; c += 2) mx = max3f(mx, x[c], x[c + 1]);
-        mx = fmaxf(mx, x[127]) * sl2;
-      } else {
-        mx = x[0];
-#pragma unroll
-        for (int c = 1; c < 127; c += 2) mx = min3f(mx, x[c], x[c + 1]);
-        mx = fminf(mx, x[127]) * sl2;
-      }
-      // The reference max m moves only when a row's max exceeds it by more than
-      // 2^8 (log2 units): until then p = 2^(x - m) <= 256, which fp32 and bf16 hold
-      // exactly enough, and O / l stays exact because both use the same m.
-      const float m_new = fmaxf(m, mx);
-      const bool rescale = __any_sync(0xffffffffu, m_new > m + 8.f);
-      float alpha = 1.f;
-      if (rescale) {
-        alpha = ex2_approx(m - m_new);  // 0 on the first tile (m = -inf)
-        l *= alpha;
-        m = m_new;
-      }
-      const float ms = (m == -INFINITY) ? 0.f : m;
-      const float nms = -ms;
-      float rs0 = 0.f, rs1 = 0.f;
-      // p = 2^(x - m), row sum, bf16 pack, and store to TMEM 32 columns at a time so
-      // the packed words never coexist with the whole fp32 row.
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
+      for (int cc = 0; cc < D / 64; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_wait_ld();
+        reg_fence32(o);
         uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int c = ch * 32 + 2 * i;
-          float a = x[c], bb = x[c + 1];
-          if (masked) {
-            a -= ms;
-            bb -= ms;
-          } else {
-            fma2(a, bb, a, bb, sl2, sl2, nms, nms);
-          }
-          a = ex2_approx(a);
-          bb = ex2_approx(bb);
-          add2(rs0, rs1, rs0, rs1, a, bb);
-          pk[i] = pack_bf16x2(a, bb);
-        }
-        tmem_st16(tS + ch * 16, pk);
-      }
-      l += rs0 + rs1;
-      if (rescale && j > 0) {
-        // Rescale this row's partial output in TMEM; PV for this tile is issued only
-        // after the arrive below, so O is stable (S_t(j) was committed after PV_t(j-1)).
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-          tmem_wait_ld();
-          reg_fence32(o);
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            float a0, a1;
-            mul2(a0, a1, __uint_as_float(o[c]), __uint_as_float(o[c + 1]), alpha, alpha);
-            o[c] = __float_as_uint(a0);
-            o[c + 1] = __float_as_uint(a1);
-          }
-          tmem_st32(tO + cc * 32, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(BAR(L::kPFull + t));
-      FA_TRACE_EVENT(blockIdx.x == 0 && (threadIdx.x & 127) == 0, FA_FWD_TR(1 + t, j, 2));
-    }
-    if (ok && nkv[t] > 0) {
-      ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kOFinal + t), 0, abort_flag, kSiteFwdSoftmax));
-      if (ok) {
-        tc_fence_after();
-        const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-        const bool row_ok = row_g < p.N;
-        uint16_t* orow = p.out + ((static_cast<size_t>(b) * p.N + row_g) * p.H + h) * D;
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-          tmem_wait_ld();
-          reg_fence32(o);
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c)
-            pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l,
-                                __uint_as_float(o[2 * c + 1]) * inv_l);
-          if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-          }
-        }
+        for (int c = 0; c < 16; ++c)
+          pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
         if (row_ok) {
-          const float lse = (l > 0.f) ? (m + __log2f(l)) * 0.69314718055994531f : -INFINITY;
-          p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + row_g] = lse;
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
         }
+      }
+      if (row_ok && half == 0) {
+        const float lse = (lt > 0.f) ? (m[t] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+        p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + row_g] = lse;
       }
     }
   }
