@@ -274,6 +274,29 @@ __global__ void timeout_probe_kernel(long long limit) {
   }
 }
 
+// Scratch for fa_bwd_noalloc, for callers that cannot allocate device memory: a
+// fixed-size array in the library's own device image (held by every GPU while the
+// library is loaded). Host code must not use the symbol as a pointer; the device
+// address is looked up per device with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on device `dev` (resolved on first use, with
+// `dev` current: the caller's current device).
+fa_status noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_bwd_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "fa_bwd_noalloc: cudaGetSymbolAddress(scratch)");
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return FA_OK;
+}
+
 __global__ void exp2_poly_kernel(const float* x, float* y, int n) {
   const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 2;
   if (i >= n) return;
@@ -368,6 +391,29 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, c
                  int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
   return fa_bwd_profiled(q, k, v, out, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, workspace,
                          workspace_bytes, stream, nullptr, nullptr);
+}
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* out,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, int causal, float scale, void* stream) {
+  if (B < 0 || H < 0 || N < 0)
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd_noalloc: negative size B=%d H=%d N=%d", B, H, N);
+  if (d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "fa_bwd_noalloc: head dim %d not supported (64 or 128)", d);
+  if (B == 0 || H == 0 || N == 0) return FA_OK;
+  const size_t need = fa::bwd_ws_layout(B, H, N, d).total;
+  if (need > FA_BWD_NOALLOC_SCRATCH_BYTES)
+    return fail(FA_ERR_WORKSPACE,
+                "fa_bwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
+                "scratch holds %u; call fa_bwd with a caller-provided workspace instead",
+                need, FA_BWD_NOALLOC_SCRATCH_BYTES);
+  int dev = 0;
+  fa_status st = current_device(&dev, nullptr);
+  if (st != FA_OK) return st;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(dev, &scratch)) != FA_OK) return st;
+  return fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, scratch,
+                FA_BWD_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 size_t fa_decode_workspace_size(int B, int H, int Ncap, int d) {

@@ -42,6 +42,9 @@ _SIGNATURES = {
                                  _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
                                  _c_int, _c_int, _c_int, _c_float, _c_void_p, _c_size_t,
                                  _c_void_p, _c_void_p, _c_void_p]),
+    "fa_bwd_noalloc": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
+                                _c_int, _c_int, _c_int, _c_float, _c_void_p]),
     "fa_decode_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
     "fa_decode": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                            _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,

@@ -101,6 +101,36 @@ fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const voi
                           size_t workspace_bytes, void* stream, void* main_start,
                           void* main_stop);
 
+/*
+ * fa_bwd for callers that cannot allocate device memory. Some callers have no way
+ * to hand this library a workspace: a host runtime that reserved all device memory
+ * at start-up and refuses later allocations, plugin or interpreter code that has
+ * no access to the application's allocator, or a latency-critical loop that must
+ * not call an allocator (which may synchronise the device). This entry point takes
+ * the same inputs and outputs as fa_bwd, minus the workspace, and uses a scratch
+ * array that lives inside the library instead. The paper has no counterpart to
+ * this call; it only exists for such callers.
+ *
+ * Limits and behaviour:
+ *  - The scratch is a fixed 32 MiB array (FA_BWD_NOALLOC_SCRATCH_BYTES) that every
+ *    GPU holds for as long as the library is loaded. Problems whose workspace
+ *    (fa_bwd_workspace_size) exceeds it are rejected with FA_ERR_WORKSPACE before
+ *    anything is launched; use fa_bwd with your own workspace for those.
+ *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine.
+ *  - The first call on each device looks up the scratch array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call before
+ *    any stream capture.
+ *  - All calls on a device share the one scratch array, which keeps whatever the
+ *    last call left in it (the backward re-initialises what it needs). Two calls
+ *    whose executions overlap on the GPU (different streams, no ordering between
+ *    them) race on the scratch and give wrong gradients: order them on one stream
+ *    or with events.
+ */
+#define FA_BWD_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* out,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int N, int d, int causal, float scale, void* stream);
+
 /* Bytes of device workspace fa_decode needs (split partials); may be 0. Depends on
  * the current device's SM count, so query it on the device that will run. */
 size_t fa_decode_workspace_size(int B, int H, int Ncap, int d);
