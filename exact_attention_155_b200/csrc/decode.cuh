@@ -29,6 +29,15 @@ namespace cg = cooperative_groups;
 
 constexpr int kDecodeMaxSplits = 8;  // CTAs per (batch, head): one portable cluster
 
+// Row steps per thread whose K and V loads are issued before any is consumed.
+#ifndef FA_DECODE_STEPS_IN_FLIGHT
+#define FA_DECODE_STEPS_IN_FLIGHT 4
+#endif
+// Target CTAs per SM when choosing the number of splits (one wave at 7 per SM).
+#ifndef FA_DECODE_CTAS_PER_SM
+#define FA_DECODE_CTAS_PER_SM 6
+#endif
+
 struct DecodeParams {
   const uint16_t* q;      // [B, 1, H, d]
   uint16_t* k_cache;      // [B, Ncap, H, d]
@@ -73,10 +82,10 @@ __device__ __forceinline__ void online_merge(float& m, float& l, float (&o)[8], 
 // memory (distributed shared memory), so the whole step is a single launch with no
 // global workspace.
 template <int D>
-__global__ void __launch_bounds__(128, 8) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
   constexpr int LPR = D / 8;     // lanes per cache row (16 bytes each)
   constexpr int RPW = 32 / LPR;  // rows per warp per step
-  constexpr int U = 4;           // steps whose loads are issued together
+  constexpr int U = FA_DECODE_STEPS_IN_FLIGHT;  // steps whose loads are issued together
   constexpr int RSTEP = 4 * RPW; // rows per CTA per step
   __shared__ float s_warp[4][D + 2];   // per-warp partial: o[D], m, l
   __shared__ float s_part[8][D + 2];   // leader only: per-CTA partials of the cluster

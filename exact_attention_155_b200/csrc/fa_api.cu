@@ -247,7 +247,7 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
 // so the grid is about one wave (6 CTAs per SM), with at least 64 keys per CTA.
 int decode_splits(int B, int H, int Ncap, int sms, int* chunk_out) {
   const long long heads = static_cast<long long>(B) * H;
-  const long long want = (static_cast<long long>(sms) * 6 + heads - 1) / std::max(1LL, heads);
+  const long long want = (static_cast<long long>(sms) * FA_DECODE_CTAS_PER_SM + heads - 1) / std::max(1LL, heads);
   int ns = 1;
   while (ns < fa::kDecodeMaxSplits && ns < want && static_cast<long long>(ns) * 2 * 64 <= Ncap) ns *= 2;
   const int chunk = (Ncap + ns - 1) / ns;
