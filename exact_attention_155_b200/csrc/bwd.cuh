@@ -317,7 +317,10 @@ __global__ void __launch_bounds__(448, 1)
     }
   } else if (warp == 13) {
     // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop (the operands stay warp-uniform); elect.sync
+    // picks the lane that issues each tcgen05 instruction, and every wait result is
+    // made uniform across the warp before it steers control.
+    {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, 0, 0);  // S^T, dP^T
       constexpr uint32_t kIdKV = idesc_bf16_f32(128, D, 0, 1);   // dV (A in TMEM), dK (A K-major)
       // d = 128: dQ^T = K^T dS^T (head dim on TMEM lanes, coalesced reductions);
@@ -330,14 +333,14 @@ __global__ void __launch_bounds__(448, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
-          umma_ss(tS, sdesc_sw128(sK + koff, 16, 1024), sdesc_sw128(sQ + koff, 16, 1024), kIdS,
+          umma_ss_w(tS, sdesc_sw128(sK + koff, 16, 1024), sdesc_sw128(sQ + koff, 16, 1024), kIdS,
                   kk > 0 ? 1u : 0u);
         }
-        umma_commit(BAR(L::kSFull));
+        umma_commit_w(BAR(L::kSFull));
       };
-      bool ok = wait_bar(BAR(L::kKVFull), 0, abort_flag, kSiteBwdMma);
+      bool ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kKVFull), 0, abort_flag, kSiteBwdMma));
       if (ok && niter > 0) {
-        ok = wait_bar(BAR(L::kQFull + 0), 0, abort_flag, kSiteBwdMma);
+        ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kQFull + 0), 0, abort_flag, kSiteBwdMma));
         if (ok) {
           tc_fence_after();
           issue_st(0);
@@ -353,64 +356,64 @@ __global__ void __launch_bounds__(448, 1)
         // dP^T(n) = V dO_n^T, into the columns dQ(n-1) used once they were read out. It
         // does not need P(n), so the dS pass can start as soon as P(n) is done.
         if (n > 0) {
-          if (!(ok = wait_bar(BAR(L::kDQFree), (n - 1) & 1, abort_flag, kSiteBwdMma))) break;
+          if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDQFree), (n - 1) & 1, abort_flag, kSiteBwdMma)))) break;
         }
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 0));
-        if (!(ok = wait_bar(BAR(L::kDOFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 0));
+        if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDOFull), n & 1, abort_flag, kSiteBwdMma)))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
-          umma_ss(tDP, sdesc_sw128(sV + koff, 16, 1024), sdesc_sw128(sdO + koff, 16, 1024), kIdS,
+          umma_ss_w(tDP, sdesc_sw128(sV + koff, 16, 1024), sdesc_sw128(sdO + koff, 16, 1024), kIdS,
                   kk > 0 ? 1u : 0u);
         }
-        umma_commit(BAR(L::kDPFull));
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 1));
+        umma_commit_w(BAR(L::kDPFull));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 1));
         // dV += P^T dO_n
-        if (!(ok = wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma))) break;
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 2));
+        if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma)))) break;
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 2));
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
+          umma_ts_w(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
                   (n > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(BAR(L::kDOEmpty));
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 3));
+        umma_commit_w(BAR(L::kDOEmpty));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 3));
         // S^T(n+1): the S columns are free once dV(n) (issued above, executed in order)
         // has read P(n); the dS pass keeps P(n) in registers.
         if (n + 1 < niter) {
-          if (!(ok = wait_bar(BAR(L::kQFull + (n + 1) % L::kQStages), ((n + 1) / L::kQStages) & 1,
-                              abort_flag, kSiteBwdMma)))
+          if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kQFull + (n + 1) % L::kQStages), ((n + 1) / L::kQStages) & 1,
+                              abort_flag, kSiteBwdMma))))
             break;
           tc_fence_after();
           issue_st(n + 1);
         }
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 4));
-        if (!(ok = wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma))) break;
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 4));
+        if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma)))) break;
         tc_fence_after();
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 5));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 5));
         // dQ_n first, so the drain reads it out of TMEM while dK(n) runs.
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           if constexpr (D == 128)
-            umma_ss(tDQ, sdesc_sw128(sK + kk * 2048, 16384, 1024),
+            umma_ss_w(tDQ, sdesc_sw128(sK + kk * 2048, 16384, 1024),
                     sdesc_sw128(sDS + kk * 2048, 16384, 1024), kIdQ, kk > 0 ? 1u : 0u);
           else
-            umma_ss(tDQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+            umma_ss_w(tDQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
                     sdesc_sw128(sK + kk * 2048, 16384, 1024), kIdQ, kk > 0 ? 1u : 0u);
         }
-        umma_commit(BAR(L::kDQFull));
+        umma_commit_w(BAR(L::kDQFull));
         // dK += dS^T Q_n
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tDK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
+          umma_ss_w(tDK, sdesc_sw128(sDS + (kk / 4) * 16384 + (kk % 4) * 32, 16, 1024),
                   sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdKV, (n > 0 || kk > 0) ? 1u : 0u);
-        umma_commit(BAR(L::kDSFree));
-        umma_commit(BAR(L::kQEmpty + s));
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(0, n, 6));
+        umma_commit_w(BAR(L::kDSFree));
+        umma_commit_w(BAR(L::kQEmpty + s));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 6));
       }
-      if (ok) umma_commit(BAR(L::kMmaDone));
-      umma_commit(BAR(L::kDrain));
+      if (ok) umma_commit_w(BAR(L::kMmaDone));
+      umma_commit_w(BAR(L::kDrain));
       drain_wait(BAR(L::kDrain), 0);
     }
   } else if (warp < 8) {

@@ -11,17 +11,19 @@
 //
 // B200 design (not the pages' A100/H100 tiling):
 //  * one CTA = one (batch, head) and 256 query rows held as two 128-row tiles;
-//  * warp 8 streams K_j and V_j (128 x d bf16) through a ring of shared-memory
+//  * the producer warp streams K_j and V_j (128 x d bf16) through a ring of shared-memory
 //    stages with TMA (128-byte swizzle) and mbarrier full/empty pairs;
-//  * warp 9 issues tcgen05.mma from one thread: S_t = Q_t K_j^T into TMEM
-//    (fp32, 128 lanes x 128 columns per tile), then O_t += P_t V_j with P_t read
-//    straight from TMEM (bf16 packed over the first 64 columns of S_t);
-//  * warps 0-7 do the softmax of one Q tile at a time (tile 0, then tile 1, per key
-//    tile): warps 0-3 take key columns 0-63 and warps 4-7 columns 64-127 of the
-//    same 128 rows (one TMEM lane per row), so all eight warps keep the exponential
-//    unit busy while the MMA warp computes the other tile's products; both halves
-//    read the whole row of scores for the row max, and each half publishes its P
-//    columns to the MMA warp as soon as they are stored;
+//  * one MMA warp per Q tile issues tcgen05.mma from one thread: S_t = Q_t K_j^T into
+//    TMEM (fp32, 128 lanes x 128 columns per tile), then O_t += P_t V_j with P_t read
+//    straight from TMEM (bf16 packed over the first 64 columns of S_t); with two
+//    issuing warps the tensor pipe keeps work queued while either one waits on a
+//    barrier or a commit;
+//  * the softmax warps (four groups of four, each group taking 32 of the 128 key
+//    columns of every row, one TMEM lane per row) work on one Q tile at a time
+//    (tile 0, then tile 1, per key tile), so all of them keep the exponential unit
+//    busy while the tensor pipe computes the other tile's products; exponentials are
+//    computed against the current reference max and redone only in the rare steps
+//    where a row grew past it; P is published to the MMA warp per 64-key half;
 //  * TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+d) O_1 [256+d,256+2d).
 #pragma once
 
@@ -41,6 +43,23 @@ struct FwdParams {
   float* lse;        // [B, H, N] fp32, natural log
 };
 
+// The softmax of a 128-row tile is split over kFwdGroups groups of four warps, each
+// taking 128 / kFwdGroups key columns of every row; more groups put more warps on the
+// exponential unit at once.
+#ifndef FA_FWD_COL_GROUPS
+#define FA_FWD_COL_GROUPS 4
+#endif
+constexpr int kFwdGroups = FA_FWD_COL_GROUPS;
+constexpr int kFwdCols = 128 / kFwdGroups;  // key columns per group
+constexpr int kFwdSoftmaxWarps = 4 * kFwdGroups;
+// Warp roles: softmax warps first, then the TMA producer, then one MMA-issuing warp
+// per Q tile. Each tile's products come from their own warp, so one warp's waits and
+// commits never leave the tensor pipe without work from the other.
+constexpr int kFwdProducerWarp = kFwdSoftmaxWarps;
+constexpr int kFwdMmaWarp = kFwdSoftmaxWarps + 1;  // tile t: kFwdMmaWarp + t
+constexpr int kFwdThreads = 32 * (kFwdSoftmaxWarps + 3);
+static_assert(kFwdGroups == 2 || kFwdGroups == 4, "2 or 4 column groups");
+
 template <int D>
 struct FwdLayout {
   static constexpr int kTileBytes = 128 * D * 2;  // one 128-row bf16 tile
@@ -55,16 +74,16 @@ struct FwdLayout {
   static constexpr int kSFull = 2 + 2 * kStages;        // [2]
   static constexpr int kPHalf = kSFull + 2;             // [2 tiles][2 key halves]
   static constexpr int kOFinal = kPHalf + 4;            // [2]
-  static constexpr int kDrain = kOFinal + 2;            // [1]
-  static constexpr int kNumBars = kDrain + 1;
-  // Exchange between the two column halves of a row: maxima [tile][half][128] fp32
-  // (exact steps only) and exp-sums [tile][half][128] fp32 (epilogue).
+  static constexpr int kDrain = kOFinal + 2;            // [2] one per MMA warp
+  static constexpr int kNumBars = kDrain + 2;
+  // Exchange between the column groups of a row: maxima [tile][group][128] fp32
+  // (exact steps only) and exp-sums [tile][group][128] fp32 (epilogue).
   static constexpr int kXMaxOff = kBarOff + kNumBars * 8;
-  static constexpr int kXSumOff = kXMaxOff + 2 * 2 * 128 * 4;
-  static constexpr int kMiscOff = kXSumOff + 2 * 2 * 128 * 4;
+  static constexpr int kXSumOff = kXMaxOff + 2 * kFwdGroups * 128 * 4;
+  static constexpr int kMiscOff = kXSumOff + 2 * kFwdGroups * 128 * 4;
   static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
-  static constexpr int kThreads = 320;
+  static constexpr int kThreads = kFwdThreads;
   static constexpr uint32_t kTmemCols = 512;
 };
 
@@ -74,6 +93,20 @@ struct FwdLayout {
 #define FA_FWD_POLY_PAIRS 0
 #endif
 constexpr int kPolyPairs = FA_FWD_POLY_PAIRS;
+
+// With FA_FWD_ALU_PACK, P is packed to bf16 on the integer pipe (pack_bf16x2_alu)
+// instead of the conversion instruction; measured about 1% slower, so off.
+#ifndef FA_FWD_ALU_PACK
+#define FA_FWD_ALU_PACK 0
+#endif
+constexpr bool kAluPack = FA_FWD_ALU_PACK != 0;
+
+// The producer asks L2 for K_j and V_j this many key tiles ahead of loading them
+// (0 = off), so the shared-memory loads that follow hit L2.
+#ifndef FA_FWD_L2_PREFETCH
+#define FA_FWD_L2_PREFETCH 0
+#endif
+constexpr int kL2Prefetch = FA_FWD_L2_PREFETCH;
 
 // Site ids for timeout reports.
 enum : unsigned int { kSiteFwdProducer = 0x101, kSiteFwdMma = 0x102, kSiteFwdSoftmax = 0x103 };
@@ -102,10 +135,10 @@ __device__ __forceinline__ float row_min128(const float (&x)[64], const float (&
 }
 
 // Trace slot of (role, key tile, event) for the traced CTA (block 0).
-#define FA_FWD_TR(role, j, e) ((((role) * 128 + ((j) & 127)) * 8) + (e))
+#define FA_FWD_TR(role, j, e) ((((role) * 128 + ((j) & 127)) * 16) + (e))
 
 template <int D, bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using L = FwdLayout<D>;
@@ -146,15 +179,17 @@ __global__ void __launch_bounds__(320, 1)
     for (int t = 0; t < 2; ++t) {
       mbar_init(BAR(L::kQFull + t), 1);
       mbar_init(BAR(L::kSFull + t), 1);
-      mbar_init(BAR(L::kPHalf + 2 * t + 0), 128);
-      mbar_init(BAR(L::kPHalf + 2 * t + 1), 128);
+      // One arrival per softmax thread whose columns fall in the key half.
+      mbar_init(BAR(L::kPHalf + 2 * t + 0), 64 * kFwdGroups);  // keys 0-63
+      mbar_init(BAR(L::kPHalf + 2 * t + 1), 64 * kFwdGroups);  // keys 64-127
       mbar_init(BAR(L::kOFinal + t), 1);
     }
     for (int s = 0; s < L::kStages; ++s) {
       mbar_init(BAR(L::kKVFull + s), 1);
-      mbar_init(BAR(L::kKVEmpty + s), 1);
+      mbar_init(BAR(L::kKVEmpty + s), 2);  // one arrival per MMA warp
     }
-    mbar_init(BAR(L::kDrain), 1);
+    mbar_init(BAR(L::kDrain + 0), 1);
+    mbar_init(BAR(L::kDrain + 1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -167,7 +202,7 @@ __global__ void __launch_bounds__(320, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 8) {
+  if (warp == kFwdProducerWarp) {
     // ------------------------------------------------------------- TMA producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -181,8 +216,17 @@ __global__ void __launch_bounds__(320, 1)
                       row0[t], b);
       }
       int it = 0;
+      if (kL2Prefetch > 0)
+        for (int j = 0; j < kL2Prefetch && j < nkv_max; ++j)
+          for (int kv = 0; kv < 2; ++kv)
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_prefetch_l2_4d(kv ? &tmV : &tmK, bx * 64, h, j * 128, b);
       for (int j = 0; j < nkv_max; ++j) {
         bool stop = false;
+        if (kL2Prefetch > 0 && j + kL2Prefetch < nkv_max)
+          for (int kv = 0; kv < 2; ++kv)
+            for (int bx = 0; bx < D / 64; ++bx)
+              tma_prefetch_l2_4d(kv ? &tmV : &tmK, bx * 64, h, (j + kL2Prefetch) * 128, b);
         for (int kv = 0; kv < 2; ++kv) {
           const int s = it % L::kStages;
           const uint32_t ph = (it / L::kStages) & 1;
@@ -190,7 +234,7 @@ __global__ void __launch_bounds__(320, 1)
             stop = true;
             break;
           }
-          FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(3, j, kv));
+          FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(9, j, kv));
           mbar_arrive_expect_tx(BAR(L::kKVFull + s), L::kTileBytes);
           const CUtensorMap* m = kv ? &tmV : &tmK;
           for (int bx = 0; bx < D / 64; ++bx)
@@ -206,119 +250,124 @@ __global__ void __launch_bounds__(320, 1)
       for (int t = 0; t < 2; ++t)
         if (nkv[t] > 0) drain_wait(BAR(L::kQFull + t), 0);
     }
-  } else if (warp == 9) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+  } else if (warp == kFwdMmaWarp || warp == kFwdMmaWarp + 1) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp kFwdMmaWarp + t issues every product of Q tile t, from one thread:
+    // S_t = Q_t K_j^T into TMEM columns [128 t, 128 t + 128), then O_t += P_t V_j with
+    // P_t read back from the same columns (bf16, two keys per column), in two key
+    // halves so the first half's products start while the softmax warps finish the
+    // second. A ring stage is free once both warps have arrived on its empty
+    // barrier: a warp that reads the stage commits after its last product on it, a
+    // warp that does not (its tile ended earlier) arrives once the stage is loaded,
+    // which keeps both arrivals in the phase of that load. The whole warp runs the
+    // loop (its operands stay warp-uniform) and elect.sync picks the issuing lane;
+    // every wait result is made uniform across the warp before it steers control.
+    const int t = warp - kFwdMmaWarp;
+    {
       constexpr uint32_t kIdQK = idesc_bf16_f32(128, 128, 0, 0);
       constexpr uint32_t kIdPV = idesc_bf16_f32(128, D, 0, 1);
+      const uint32_t sQt = sQ + t * L::kTileBytes;
+      const uint32_t tS = tmem + t * 128;
+      const uint32_t tO = tmem + 256 + t * D;
       bool ok = true;
-      auto issue_qk = [&](int t, int s) {
-        const uint32_t dt = tmem + t * 128;
+      auto issue_qk = [&](int s) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t koff = (kk / 4) * 16384 + (kk % 4) * 32;
-          const uint64_t ad = sdesc_sw128(sQ + t * L::kTileBytes + koff, 16, 1024);
+          const uint64_t ad = sdesc_sw128(sQt + koff, 16, 1024);
           const uint64_t bd = sdesc_sw128(sKV + s * L::kTileBytes + koff, 16, 1024);
-          umma_ss(dt, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
+          umma_ss_w(tS, ad, bd, kIdQK, kk > 0 ? 1u : 0u);
         }
       };
       // O_t += P_t V for keys [64*half, 64*half + 64) of the tile.
-      auto issue_pv_half = [&](int t, int s, int half, bool acc) {
-        const uint32_t dt = tmem + 256 + t * D;
-        const uint32_t at = tmem + t * 128;
+      auto issue_pv_half = [&](int s, int half, bool acc) {
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = half * 4 + k4;
           const uint64_t bd = sdesc_sw128(sKV + s * L::kTileBytes + kk * 2048, 16384, 1024);
-          umma_ts(dt, at + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts_w(tO, tS + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
         }
       };
-      for (int t = 0; t < 2 && ok; ++t)
-        if (nkv[t] > 0) ok = wait_bar(BAR(L::kQFull + t), 0, abort_flag, kSiteFwdMma);
-      if (ok) {
-        // S_t for key tile 0 (ring load 0).
-        ok = wait_bar(BAR(L::kKVFull + 0), 0, abort_flag, kSiteFwdMma);
+      const int n = nkv[t];
+      if (n > 0) {
+        ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kQFull + t), 0, abort_flag, kSiteFwdMma) &&
+                                         wait_bar(BAR(L::kKVFull + 0), 0, abort_flag, kSiteFwdMma));
         if (ok) {
           tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (nkv[t] == 0) continue;
-            issue_qk(t, 0);
-            umma_commit(BAR(L::kSFull + t));
-          }
-          umma_commit(BAR(L::kKVEmpty + 0));
+          issue_qk(0);
+          umma_commit_w(BAR(L::kSFull + t));
+          umma_commit_w(BAR(L::kKVEmpty + 0));
         }
       }
-      for (int j = 0; j < nkv_max && ok; ++j) {
+      for (int j = 0; j < n && ok; ++j) {
         const int iv = 2 * j + 1, ik = 2 * j + 2;
         const int sv = iv % L::kStages, sk = ik % L::kStages;
-        if (!wait_bar(BAR(L::kKVFull + sv), (iv / L::kStages) & 1, abort_flag, kSiteFwdMma)) {
+        ok = __all_sync(0xffffffffu,
+                        wait_bar(BAR(L::kKVFull + sv), (iv / L::kStages) & 1, abort_flag, kSiteFwdMma));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 10 * t));
+        if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kPHalf + 2 * t + 0), j & 1, abort_flag, kSiteFwdMma));
+        if (!ok) break;
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 1 + 4 * t));
+        tc_fence_after();
+        issue_pv_half(sv, 0, j > 0);
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 2 + 4 * t));
+        if (!__all_sync(0xffffffffu, wait_bar(BAR(L::kPHalf + 2 * t + 1), j & 1, abort_flag, kSiteFwdMma))) {
           ok = false;
           break;
         }
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(0, j, 0));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 3 + 4 * t));
         tc_fence_after();
-        bool k_next = false;
-        for (int t = 0; t < 2; ++t) {
-          if (j >= nkv[t]) continue;
-          // P_t arrives in two key halves; the first half's products start while the
-          // softmax warpgroup is still exponentiating the second half.
-          if (!wait_bar(BAR(L::kPHalf + 2 * t + 0), j & 1, abort_flag, kSiteFwdMma)) {
-            ok = false;
-            break;
-          }
-          FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(0, j, 1 + 2 * t));
-          tc_fence_after();
-          issue_pv_half(t, sv, 0, j > 0);
-          if (!wait_bar(BAR(L::kPHalf + 2 * t + 1), j & 1, abort_flag, kSiteFwdMma)) {
+        issue_pv_half(sv, 1, j > 0);
+        const bool more = j + 1 < n;
+        if (more) {
+          if (!__all_sync(0xffffffffu,
+                          wait_bar(BAR(L::kKVFull + sk), (ik / L::kStages) & 1, abort_flag, kSiteFwdMma))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          issue_pv_half(t, sv, 1, j > 0);
-          if (j + 1 < nkv[t]) {
-            if (!k_next) {
-              if (!wait_bar(BAR(L::kKVFull + sk), (ik / L::kStages) & 1, abort_flag,
-                            kSiteFwdMma)) {
-                ok = false;
-                break;
-              }
-              tc_fence_after();
-              k_next = true;
-            }
-            issue_qk(t, sk);
-            umma_commit(BAR(L::kSFull + t));
-          } else {
-            umma_commit(BAR(L::kOFinal + t));
-          }
-          FA_TRACE_EVENT(blockIdx.x == 0, FA_FWD_TR(0, j, 2 + 2 * t));
+          issue_qk(sk);
+          umma_commit_w(BAR(L::kSFull + t));
+        } else {
+          umma_commit_w(BAR(L::kOFinal + t));
         }
-        if (!ok) break;
-        umma_commit(BAR(L::kKVEmpty + sv));
-        if (k_next) umma_commit(BAR(L::kKVEmpty + sk));
+        umma_commit_w(BAR(L::kKVEmpty + sv));
+        if (more) umma_commit_w(BAR(L::kKVEmpty + sk));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 4 + 4 * t));
+      }
+      // Ring loads after this tile's last key tile: K_n, V_n, ..., V_(nkv_max - 1).
+      for (int x = 2 * n; x < 2 * nkv_max && ok; ++x) {
+        const int s = x % L::kStages;
+        ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kKVFull + s), (x / L::kStages) & 1, abort_flag, kSiteFwdMma));
+        if (ok && lane == 0) mbar_arrive(BAR(L::kKVEmpty + s));
       }
       // Let every issued MMA finish before TMEM can be released.
-      umma_commit(BAR(L::kDrain));
-      drain_wait(BAR(L::kDrain), 0);
+      umma_commit_w(BAR(L::kDrain + t));
+      drain_wait(BAR(L::kDrain + t), 0);
     }
   } else {
     // ------------------------------------------------------------ softmax warps
-    // All eight warps work on one Q tile at a time (tile 0, then tile 1, for every
-    // key tile j): warpgroup `half` takes key columns [64*half, 64*half + 64) of each
-    // of the 128 rows, so the exponential unit is shared by two warps per SM
-    // sub-partition while the MMA warp runs the other tile's products. The two
-    // halves of a row both read the whole row of scores for the row max, and add
-    // their exp-sums through shared memory at the end; P is published to the MMA
-    // warp per half.
-    const int half = warp >> 2;
-    const int wq = warp & 3;
+    // The softmax warps work on one Q tile at a time (tile 0, then tile 1, for every
+    // key tile j). Group g (warps 4g..4g+3) takes key columns [g*C, g*C + C),
+    // C = 128 / kFwdGroups, of each of the 128 rows (one TMEM lane per row), so all
+    // softmax warps share the exponential unit on one tile while the MMA warp runs
+    // the other tile's products. Column groups of a row meet in shared memory only
+    // on exact steps (row maxima) and at the end (exp-sums).
+    constexpr int C = kFwdCols;
+    constexpr int NTQ = 32 * kFwdGroups;  // threads of one lane quarter (named barriers)
+    const int grp = warp >> 2;
+    const int wq = warp & 3;  // TMEM lane quarter this warp may access
     const int r = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    // Named barriers of this lane quarter: 1-4 for the per-tile vote and max exchange,
+    // 5-8 for the epilogue's exp-sum exchange (0 is __syncthreads).
+    const int kBarVote = 1 + wq, kBarEpi = 5 + wq;
     const float sl2 = p.scale_log2;
     float* xmax = reinterpret_cast<float*>(smem + L::kXMaxOff);
     float* xsum = reinterpret_cast<float*>(smem + L::kXSumOff);
-    const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
+    const bool tr = blockIdx.x == 0 && grp == 0 && lane == 0;  // group 0, one thread per warp
     float m[2] = {-INFINITY, -INFINITY};  // running row max per tile (log2 units)
-    float l[2] = {0.f, 0.f};              // running exp-sum over this half's columns
+    float l[2] = {0.f, 0.f};              // running exp-sum over this group's columns
     bool ok = true;
     for (int j = 0; j < nkv_max && ok; ++j) {
 #pragma unroll
@@ -329,48 +378,43 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t tO = tmem + 256 + t * D + lane_off;
         const bool w_ok = __all_sync(0xffffffffu,
                                      wait_bar(BAR(L::kSFull + t), j & 1, abort_flag, kSiteFwdSoftmax));
-        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 0));
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 0));
         tc_fence_after();
-        uint32_t s0[32], s1[32];
-        tmem_ld32(tS + 64 * half, s0);
-        tmem_ld32(tS + 64 * half + 32, s1);
-        tmem_wait_ld();
-        reg_fence32(s0);
-        reg_fence32(s1);
-        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 1));
-        float x[64];
+        float x[C];
+        {
+          uint32_t s0[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          x[c] = __uint_as_float(s0[c]);
-          x[32 + c] = __uint_as_float(s1[c]);
+          for (int q32 = 0; q32 < C / 32; ++q32) {
+            tmem_ld32(tS + C * grp + 32 * q32, s0);
+            tmem_wait_ld();
+            reg_fence32(s0);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) x[32 * q32 + c] = __uint_as_float(s0[c]);
+          }
         }
-        const int kbase = j * 128 + 64 * half;  // key index of column 0 of this half
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 1));
+        const int kbase = j * 128 + C * grp;  // key index of this group's column 0
         const bool masked = (CAUSAL && j * 128 == row0[t]) || (j * 128 + 128 > p.N);
         if (masked) {
           // Diagonal or tail tile: scale first, then mask to -inf.
           const int lim = CAUSAL ? min(row_g, p.N - 1) : p.N - 1;
 #pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = (kbase + c > lim) ? -INFINITY : x[c] * sl2;
+          for (int c = 0; c < C; ++c) x[c] = (kbase + c > lim) ? -INFINITY : x[c] * sl2;
         }
         // x holds raw scores (unmasked tile) or scaled, masked scores (masked tile).
-        // exps(ms, mx_out): p = 2^(x*sl2 - ms) (resp. 2^(x - ms)) for this half's 64
-        // columns, their sum, bf16 P into TMEM, and this half's max of the scaled
-        // scores computed alongside on the ALU (8 independent accumulators).
+        // exps(ms): p = 2^(x*sl2 - ms) (resp. 2^(x - ms)) for this group's C columns,
+        // their sum into rsum, and bf16 P into TMEM.
         float rsum = 0.f;
-        auto exps = [&](float ms, float& mx_out) {
+        auto exps = [&](float ms) {
           const float nms = -ms;
           float rs[4] = {0.f, 0.f, 0.f, 0.f};
-          float acc[8];
 #pragma unroll
-          for (int a8 = 0; a8 < 8; ++a8) acc[a8] = -INFINITY;
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
+          for (int ch = 0; ch < C / 32; ++ch) {
             uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int c = ch * 32 + 2 * i;
               float a = x[c], bb = x[c + 1];
-              acc[i & 7] = max3f(acc[i & 7], a, bb);
               if (masked) {
                 a -= ms;
                 bb -= ms;
@@ -384,64 +428,69 @@ __global__ void __launch_bounds__(320, 1)
                 bb = ex2_approx(bb);
               }
               add2(rs[2 * (i & 1)], rs[2 * (i & 1) + 1], rs[2 * (i & 1)], rs[2 * (i & 1) + 1], a, bb);
-              pk[i] = pack_bf16x2(a, bb);
+              pk[i] = kAluPack ? pack_bf16x2_alu(a, bb) : pack_bf16x2(a, bb);
             }
-            tmem_st16(tS + 32 * half + ch * 16, pk);
+            tmem_st16(tS + (C / 2) * grp + ch * 16, pk);  // P: two keys per 32-bit column
           }
-          float mxr = fmaxf(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], max3f(acc[5], acc[6], acc[7])));
-          mx_out = masked ? mxr : mxr * sl2;
           rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
         };
-        // Fast path: exponentiate against the current reference max while computing
-        // this half's max; if no row of the tile grew past the reference by more than
-        // 2^8, P is final (p <= 256 stays exact enough in fp32 and bf16, and O / l stays
-        // exact because both use the same reference).
-        // The fast/exact choice is uniform over all 256 softmax threads (j and the
-        // scale's sign are), so every thread reaches the same named barriers; an
-        // abort is folded into the vote and forces the exact path, which ends it.
+        // Fast path: exponentiate against the current reference max. If this group's
+        // exponentials of every row sum to at most 256, none of them exceeds 2^8, so P
+        // is final (p <= 256 stays exact enough in fp32 and bf16, and O / l stays exact
+        // because both use the same reference). The check costs one compare on a sum
+        // that is needed anyway, instead of a running max over every score. The choice
+        // is made per TMEM lane quarter: the groups of a row are the G warps of one
+        // quarter (same SMSP), and rows of different quarters never exchange anything.
+        // It is uniform over those warps (j and the scale's sign are), so they all reach
+        // the same named barriers; an abort is folded into the vote and forces the exact
+        // path, which ends it. A NaN or infinite sum fails the compare and also goes
+        // exact.
         bool exact = (j == 0) || !(sl2 >= 0.f);
-        float mx_half = -INFINITY;
         if (!exact) {
-          exps(m[t], mx_half);
-          exact = named_bar_or(1, 256, !w_ok || !(mx_half <= m[t] + 8.f));
+          exps(m[t]);
+          exact = named_bar_or(kBarVote, NTQ, !w_ok || !(rsum <= 256.f));
           if (!exact) l[t] += rsum;
         }
         if (exact) {
-          // Exact path (first tile, negative scale, a grown row, or an abort): the two
-          // halves exchange their maxima, move the reference, rescale O, and (re)do
-          // the exponentials.
-          if (mx_half == -INFINITY) {
+          // Exact path (first tile, negative scale, a grown row, or an abort): the
+          // column groups exchange their maxima, move the reference, rescale O, and
+          // (re)do the exponentials.
+          float mx_grp;
+          {
             float acc[8];
+            const bool up = masked || sl2 >= 0.f;
 #pragma unroll
-            for (int a8 = 0; a8 < 8; ++a8) acc[a8] = (sl2 >= 0.f || masked) ? -INFINITY : INFINITY;
-            if (masked || sl2 >= 0.f) {
+            for (int a8 = 0; a8 < 8; ++a8) acc[a8] = up ? -INFINITY : INFINITY;
+            if (up) {
 #pragma unroll
-              for (int c = 0; c < 64; c += 2) acc[(c >> 1) & 7] = max3f(acc[(c >> 1) & 7], x[c], x[c + 1]);
+              for (int c = 0; c < C; c += 2) acc[(c >> 1) & 7] = max3f(acc[(c >> 1) & 7], x[c], x[c + 1]);
               const float mxr = fmaxf(max3f(acc[0], acc[1], acc[2]), max3f(acc[3], acc[4], max3f(acc[5], acc[6], acc[7])));
-              mx_half = masked ? mxr : mxr * sl2;
+              mx_grp = masked ? mxr : mxr * sl2;
             } else {
 #pragma unroll
-              for (int c = 0; c < 64; c += 2) acc[(c >> 1) & 7] = min3f(acc[(c >> 1) & 7], x[c], x[c + 1]);
-              mx_half = fminf(min3f(acc[0], acc[1], acc[2]), min3f(acc[3], acc[4], min3f(acc[5], acc[6], acc[7]))) * sl2;
+              for (int c = 0; c < C; c += 2) acc[(c >> 1) & 7] = min3f(acc[(c >> 1) & 7], x[c], x[c + 1]);
+              mx_grp = fminf(min3f(acc[0], acc[1], acc[2]), min3f(acc[3], acc[4], min3f(acc[5], acc[6], acc[7]))) * sl2;
             }
           }
-          float* xm = xmax + t * 256;
-          xm[half * 128 + r] = mx_half;
-          ok = named_bar_and(1, 256, w_ok);
+          float* xm = xmax + t * (128 * kFwdGroups);
+          xm[grp * 128 + r] = mx_grp;
+          ok = named_bar_and(kBarVote, NTQ, w_ok);
           if (!ok) break;
-          const float mx = fmaxf(mx_half, xm[(half ^ 1) * 128 + r]);
+          float mx = mx_grp;
+#pragma unroll
+          for (int g2 = 0; g2 < kFwdGroups; ++g2) mx = fmaxf(mx, xm[g2 * 128 + r]);
           const float m_new = fmaxf(m[t], mx);
           if (__any_sync(0xffffffffu, m_new > m[t] + 8.f)) {
             const float alpha = ex2_approx(m[t] - m_new);  // 0 on the first tile (m = -inf)
             l[t] *= alpha;
             m[t] = m_new;
             if (j > 0) {
-              // Rescale this half of the row's partial output before this tile's
-              // products accumulate into it (PV_t(j-1) completed before S_t(j)).
+              // Rescale this group's D/G columns of the row's partial output before this
+              // tile's products accumulate into it (PV_t(j-1) completed before S_t(j)).
 #pragma unroll
-              for (int cc = 0; cc < D / 32; ++cc) {
+              for (int cc = 0; cc < D / kFwdGroups / 16; ++cc) {
                 uint32_t o[16];
-                tmem_ld16(tO + half * (D / 2) + cc * 16, o);
+                tmem_ld16(tO + grp * (D / kFwdGroups) + cc * 16, o);
                 tmem_wait_ld();
                 reg_fence16(o);
 #pragma unroll
@@ -451,62 +500,63 @@ __global__ void __launch_bounds__(320, 1)
                   o[c] = __float_as_uint(a0);
                   o[c + 1] = __float_as_uint(a1);
                 }
-                tmem_st16(tO + half * (D / 2) + cc * 16, o);
+                tmem_st16(tO + grp * (D / kFwdGroups) + cc * 16, o);
               }
             }
           }
           // The exchange slots are reused at the next exact step of this tile only
           // after every thread has read them.
-          named_bar_sync(1, 256);
-          float unused;
-          exps(m[t] == -INFINITY ? 0.f : m[t], unused);
+          named_bar_sync(kBarVote, NTQ);
+          exps(m[t] == -INFINITY ? 0.f : m[t]);
           l[t] += rsum;
         }
-        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 4));
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 2));
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(BAR(L::kPHalf + 2 * t + half));
-        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + t, j, 2));
+        mbar_arrive(BAR(L::kPHalf + 2 * t + (grp * C) / 64));
+        FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 3));
       }
     }
-    // Epilogue per tile: O / l and the LSE. Each half writes its D/2 output columns.
+    // Epilogue per tile: O / l and the LSE. Each group writes its D/G output columns.
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       if (nkv[t] == 0) continue;  // uniform over the CTA
       // Every softmax thread reaches the barrier below, aborted or not; the AND
-      // carries the abort so all 256 threads leave together.
+      // carries the abort so all of them leave together.
       bool w_ok = ok;
       if (w_ok) w_ok = wait_bar(BAR(L::kOFinal + t), 0, abort_flag, kSiteFwdSoftmax);
       w_ok = __all_sync(0xffffffffu, w_ok);
-      float* xs = xsum + t * 256;
-      xs[half * 128 + r] = l[t];
-      ok = named_bar_and(2, 256, w_ok);
+      float* xs = xsum + t * (128 * kFwdGroups);
+      xs[grp * 128 + r] = l[t];
+      ok = named_bar_and(kBarEpi, NTQ, w_ok);
       if (!ok) continue;
-      const float lt = l[t] + xs[(half ^ 1) * 128 + r];
+      float lt = 0.f;
+#pragma unroll
+      for (int g2 = 0; g2 < kFwdGroups; ++g2) lt += xs[g2 * 128 + r];
       tc_fence_after();
       const int row_g = row0[t] + r;
-      const uint32_t tO = tmem + 256 + t * D + lane_off + half * (D / 2);
+      constexpr int DG = D / kFwdGroups;  // output columns of this group
+      const uint32_t tO = tmem + 256 + t * D + lane_off + grp * DG;
       const float inv_l = (lt > 0.f) ? 1.f / lt : 0.f;
       const bool row_ok = row_g < p.N;
-      uint16_t* orow = p.out + ((static_cast<size_t>(b) * p.N + row_g) * p.H + h) * D + half * (D / 2);
+      uint16_t* orow = p.out + ((static_cast<size_t>(b) * p.N + row_g) * p.H + h) * D + grp * DG;
 #pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
+      for (int cc = 0; cc < DG / 16; ++cc) {
+        uint32_t o[16];
+        tmem_ld16(tO + cc * 16, o);
         tmem_wait_ld();
-        reg_fence32(o);
-        uint32_t pk[16];
+        reg_fence16(o);
+        uint32_t pk[8];
 #pragma unroll
-        for (int c = 0; c < 16; ++c)
+        for (int c = 0; c < 8; ++c)
           pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
         if (row_ok) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            dst[v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+          uint4* dst = reinterpret_cast<uint4*>(orow + cc * 16);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
         }
       }
-      if (row_ok && half == 0) {
+      if (row_ok && grp == 0) {
         const float lse = (lt > 0.f) ? (m[t] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
         p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + row_g] = lse;
       }

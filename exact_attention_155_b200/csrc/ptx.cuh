@@ -119,6 +119,15 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
       : "memory");
 }
+// Bring a tile of a tensor into L2 without writing shared memory (no completion to
+// wait for; out-of-range boxes are dropped by the hardware).
+__device__ __forceinline__ void tma_prefetch_l2_4d(const CUtensorMap* map, int c0, int c1, int c2,
+                                                   int c3) {
+  asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -168,6 +177,37 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
                    bar)
                : "memory");
+}
+
+// Warp-wide forms of the three issue instructions above: all 32 lanes of a converged
+// warp execute the call (so the operands stay warp-uniform) and elect.sync picks the
+// one lane that issues.
+__device__ __forceinline__ void umma_ss_w(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_ts_w(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_w(uint32_t bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(bar)
+      : "memory");
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
@@ -262,6 +302,17 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// The same packing on the integer pipe (no conversion unit): round to nearest with
+// ties away from zero by adding half a bf16 ulp to the fp32 bit pattern (a carry
+// into the exponent is the correct rounding), then keep the two high halves with one
+// byte permute. Differs from round-to-nearest-even only on exact ties. For finite
+// inputs below the bf16 overflow threshold, which is all the softmax produces.
+__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
+  const uint32_t a = __float_as_uint(lo) + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) + 0x8000u;
+  return __byte_perm(a, b, 0x7632);  // bytes 2,3 of a, then bytes 2,3 of b
+}
+
 // Packed fp32x2 arithmetic (sm_100): two lanes of work per instruction.
 __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
                                      float c0, float c1) {
@@ -315,8 +366,10 @@ __device__ __forceinline__ void exp2_poly2(float& a, float& b) {
   fma2(pa, pb, fa, fb, c3, c3, c2, c2);
   fma2(pa, pb, pa, pb, fa, fb, c1, c1);
   fma2(pa, pb, pa, pb, fa, fb, 1.f, 1.f);
-  a = __uint_as_float(__float_as_uint(pa) + ((__float_as_uint(ta) - 0x4B400000u) << 23));
-  b = __uint_as_float(__float_as_uint(pb) + ((__float_as_uint(tb) - 0x4B400000u) << 23));
+  // The low mantissa bits of t hold j + 2^22; shifted into the exponent field the
+  // 2^22 term leaves the 32-bit word, so (bits(t) << 23) adds exactly j to the exponent.
+  a = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
+  b = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
 }
 
 __device__ __forceinline__ void red_add_f32(float* addr, float v) {
