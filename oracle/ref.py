@@ -36,6 +36,15 @@ Readings taken where the pages are silent (each is also listed in the design not
   cache_seqlens[b] + 1 rows; without it, it covers cache_seqlens[b] rows.
 * The backward is the analytic gradient of the definition (the pages only say the
   scores are recomputed, not stored).
+* Sliding window ("Flash-Attention 2/3在ms-swift中的集成与性能提升", FA3 feature list;
+  the page names the mask, not its parameters): with the query's position on the key
+  axis i' = i + (Nk - Nq), key j is visible iff i' - window_left <= j <= i' +
+  window_right; -1 leaves a side unbounded. It combines with the causal mask by AND.
+* Variable-length batches (packing, "ms-swift长文本训练优化，Flash-Attention显存省一半"
+  sections 4.2 and 5.1): tokens of B sequences are packed into [total, H, d] and
+  sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]); each sequence is an
+  independent attention problem (nothing is attended across sequences); the LSE is
+  laid out [H, total].
 
 Every array is numpy float64; callers convert the exact bf16 input values first.
 Large problems are processed in blocks of query rows; each block's softmax is the
@@ -51,10 +60,13 @@ import numpy as np
 __all__ = [
     "default_scale",
     "visible_mask",
+    "window_mask",
     "scores",
     "softmax_rows",
     "attention_forward",
     "attention_backward",
+    "attention_forward_varlen",
+    "attention_backward_varlen",
     "blockwise_forward",
     "merge_partials",
     "decode_step",
@@ -77,6 +89,28 @@ def visible_mask(q_pos: np.ndarray, nk: int, causal: bool, nq_total: int) -> np.
     if not causal:
         return np.ones((len(q_pos), nk), dtype=bool)
     return j <= (np.asarray(q_pos)[:, None] + (nk - nq_total))
+
+
+def window_mask(q_pos: np.ndarray, nk: int, nq_total: int, window_left: int,
+                window_right: int) -> np.ndarray:
+    """Boolean [len(q_pos), nk] sliding-window mask: key j visible to query i iff
+    i' - window_left <= j <= i' + window_right with i' = i + (nk - nq_total);
+    -1 = unbounded side."""
+    j = np.arange(nk)[None, :]
+    ip = np.asarray(q_pos)[:, None] + (nk - nq_total)
+    m = np.ones((len(q_pos), nk), dtype=bool)
+    if window_left >= 0:
+        m &= j >= ip - window_left
+    if window_right >= 0:
+        m &= j <= ip + window_right
+    return m
+
+
+def _mask(ridx, nk, causal, nq, window_left, window_right):
+    mask = visible_mask(ridx, nk, causal, nq)
+    if window_left >= 0 or window_right >= 0:
+        mask = mask & window_mask(ridx, nk, nq, window_left, window_right)
+    return mask
 
 
 def scores(qm: np.ndarray, km: np.ndarray, scale: float) -> np.ndarray:
@@ -106,7 +140,7 @@ def _resolve_scale(scale, d):
 
 
 def attention_forward(q, k, v, causal=False, scale=None, row_block=1024,
-                      heads=None, rows=None):
+                      heads=None, rows=None, window_left=-1, window_right=-1):
     """Exact attention forward, materialising S per (b, h) in query-row blocks.
 
     q: [B, Nq, H, d]; k, v: [B, Nk, H, d] (float64).
@@ -131,7 +165,7 @@ def attention_forward(q, k, v, causal=False, scale=None, row_block=1024,
         for s0 in range(0, len(row_idx), row_block):
             ridx = row_idx[s0:s0 + row_block]
             qm = q[b, ridx, h, :]
-            mask = visible_mask(ridx, Nk, causal, Nq)
+            mask = _mask(ridx, Nk, causal, Nq, window_left, window_right)
             p, l = softmax_rows(scores(qm, km, sc), mask)
             out[b, ridx, h, :] = p @ vm
             lse[b, h, ridx] = l
@@ -139,7 +173,7 @@ def attention_forward(q, k, v, causal=False, scale=None, row_block=1024,
 
 
 def attention_backward(q, k, v, dout, causal=False, scale=None, row_block=1024,
-                       heads=None):
+                       heads=None, window_left=-1, window_right=-1):
     """Analytic gradients of out = softmax(scale*Q K^T, mask) V.
 
     With P the row softmax and dO the output gradient:
@@ -169,7 +203,7 @@ def attention_backward(q, k, v, dout, causal=False, scale=None, row_block=1024,
             ridx = np.arange(r0, min(Nq, r0 + row_block))
             qm = q[b, ridx, h, :]
             dom = dout[b, ridx, h, :]
-            mask = visible_mask(ridx, Nk, causal, Nq)
+            mask = _mask(ridx, Nk, causal, Nq, window_left, window_right)
             p, _ = softmax_rows(scores(qm, km, sc), mask)
             dv_acc += p.T @ dom
             dp = dom @ vm.T
@@ -179,6 +213,50 @@ def attention_backward(q, k, v, dout, causal=False, scale=None, row_block=1024,
             dk_acc += sc * (ds.T @ qm)
         dk[b, :, h, :] = dk_acc
         dv[b, :, h, :] = dv_acc
+    return dq, dk, dv
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, causal=False, scale=None,
+                             window_left=-1, window_right=-1):
+    """Packed variable-length forward: q, k, v [total, H, d]; sequence b is tokens
+    [cu_seqlens[b], cu_seqlens[b+1]). Returns out [total, H, d] and lse [H, total]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    total, H, d = q.shape
+    out = np.full((total, H, v.shape[2]), np.nan)
+    lse = np.full((H, total), np.nan)
+    cu = [int(x) for x in cu_seqlens]
+    for b in range(len(cu) - 1):
+        s0, s1 = cu[b], cu[b + 1]
+        if s1 == s0:
+            continue
+        o, l = attention_forward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], causal=causal,
+                                 scale=scale, window_left=window_left, window_right=window_right)
+        out[s0:s1] = o[0]
+        lse[:, s0:s1] = l[0]
+    return out, lse
+
+
+def attention_backward_varlen(q, k, v, dout, cu_seqlens, causal=False, scale=None,
+                              window_left=-1, window_right=-1):
+    """Gradients of attention_forward_varlen; dq, dk, dv [total, H, d]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    dq = np.full(q.shape, np.nan)
+    dk = np.full(k.shape, np.nan)
+    dv = np.full(v.shape, np.nan)
+    cu = [int(x) for x in cu_seqlens]
+    for b in range(len(cu) - 1):
+        s0, s1 = cu[b], cu[b + 1]
+        if s1 == s0:
+            continue
+        g = attention_backward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1], dout[None, s0:s1],
+                               causal=causal, scale=scale, window_left=window_left,
+                               window_right=window_right)
+        dq[s0:s1], dk[s0:s1], dv[s0:s1] = g[0][0], g[1][0], g[2][0]
     return dq, dk, dv
 
 
