@@ -35,21 +35,50 @@
 namespace fa {
 
 struct BwdParams {
-  int B, H, N, Np;      // Np = N rounded up to a multiple of 128
+  int B, H, N, Np;      // N: sequence length (dense) or the largest one (variable length);
+                        // Np = N rounded up to a multiple of 128
   int nqt;              // Np / 128
   int head_group;       // heads scheduled together (divides B*H), for L2 reuse
+  int window_left;      // keys visible to query i: [i - window_left, i + window_right],
+  int window_right;     // -1 = unbounded on that side (causal: window_right = 0)
   float scale;          // softmax scale
   float scale_log2;     // scale * log2(e)
-  const uint16_t* out;  // forward output [B, N, H, d]
-  const uint16_t* dout; // [B, N, H, d]
-  const float* lse;     // [B, H, N] natural log
+  const int* cu_seqlens;  // NULL: dense rows (b, n); else [B + 1] token offsets
+  int total;            // variable length: tokens in the packed tensors
+  // Elements between consecutive rows (tokens) of each row-major [*, H, d] tensor.
+  long long rs_o, rs_do, rs_dq, rs_dk, rs_dv;
+  const uint16_t* out;  // forward output
+  const uint16_t* dout;
+  const float* lse;     // dense [B, H, N]; variable [H, total]; natural log
   float* dq_acc;        // [B, H, Np, d] fp32
-  float* lse2;          // [B, H, Np] log2 units (+inf on padded rows)
+  float* lse2;          // [B, H, Np] log2 units (+inf on rows past the sequence)
   float* dvec;          // [B, H, Np] rowsum(dO * O)
-  uint16_t* dq;         // [B, N, H, d]
+  uint16_t* dq;
   uint16_t* dk;
   uint16_t* dv;
 };
+
+enum : unsigned int {
+  kSiteBwdProducer = 0x201,
+  kSiteBwdMma = 0x202,
+  kSiteBwdSoftmax = 0x203,
+  kSiteBwdDrain = 0x204,
+  kSiteBwdSeqlens = 0x205,
+  kSiteBwdSmemAlign = 0x2FF
+};
+
+// First token and length of sequence b; false for an invalid cu_seqlens entry.
+__device__ __forceinline__ bool bwd_seq(const BwdParams& p, int b, long long* tok0, int* len) {
+  if (p.cu_seqlens == nullptr) {
+    *tok0 = static_cast<long long>(b) * p.N;
+    *len = p.N;
+    return true;
+  }
+  const int s0 = __ldg(p.cu_seqlens + b), s1 = __ldg(p.cu_seqlens + b + 1);
+  *tok0 = s0;
+  *len = s1 - s0;
+  return !(s0 < 0 || s1 < s0 || s1 - s0 > p.N || s1 > p.total);
+}
 
 struct BwdWorkspace {
   size_t dq_off, lse2_off, dvec_off, total;
@@ -79,11 +108,16 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   const int i = valid ? static_cast<int>(row % p.Np) : 0;
   const long long bh = valid ? row / p.Np : 0;
   const int b = static_cast<int>(bh / p.H), h = static_cast<int>(bh % p.H);
+  long long tok0 = 0;
+  int len = 0;
+  const bool seq_ok = valid && bwd_seq(p, b, &tok0, &len);
+  if (valid && !seq_ok && i == 0 && sub == 0 && h == 0) report(kDevBadInput, kSiteBwdSeqlens, b);
+  const bool real = seq_ok && i < len;
   float acc = 0.f;
-  if (valid && i < p.N) {
-    const size_t off = ((static_cast<size_t>(b) * p.N + i) * p.H + h) * D + sub * 8;
-    const uint4 o = __ldg(reinterpret_cast<const uint4*>(p.out + off));
-    const uint4 g = __ldg(reinterpret_cast<const uint4*>(p.dout + off));
+  if (real) {
+    const long long tok = tok0 + i;
+    const uint4 o = __ldg(reinterpret_cast<const uint4*>(p.out + tok * p.rs_o + h * D + sub * 8));
+    const uint4 g = __ldg(reinterpret_cast<const uint4*>(p.dout + tok * p.rs_do + h * D + sub * 8));
     const uint32_t ow[4] = {o.x, o.y, o.z, o.w}, gw[4] = {g.x, g.y, g.z, g.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -95,9 +129,12 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
   for (int o = TPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
   if (!valid) return;
   if (sub == 0) {
-    const bool real = i < p.N;
+    float lse = INFINITY;
+    if (real)
+      lse = (p.cu_seqlens != nullptr ? p.lse[static_cast<size_t>(h) * p.total + tok0 + i]
+                                     : p.lse[bh * p.N + i]) * 1.4426950408889634f;
     p.dvec[row] = real ? acc : 0.f;
-    p.lse2[row] = real ? p.lse[bh * p.N + i] * 1.4426950408889634f : INFINITY;
+    p.lse2[row] = lse;
   }
   float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D + sub * 8);
   z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -116,6 +153,9 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const BwdParams p) 
   const long long bi = row / p.H;
   const int i = static_cast<int>(bi % p.N);
   const int b = static_cast<int>(bi / p.N);
+  long long tok0 = 0;
+  int len = 0;
+  if (!bwd_seq(p, b, &tok0, &len) || i >= len) return;
   const float4* src = reinterpret_cast<const float4*>(
       p.dq_acc + ((static_cast<size_t>(b) * p.H + h) * p.Np + i) * D + sub * 8);
   const float4 a = src[0], c = src[1];
@@ -124,7 +164,7 @@ __global__ void __launch_bounds__(256) bwd_dq_convert_kernel(const BwdParams p) 
   o.y = pack_bf16x2(a.z, a.w);
   o.z = pack_bf16x2(c.x, c.y);
   o.w = pack_bf16x2(c.z, c.w);
-  *reinterpret_cast<uint4*>(p.dq + row * D + sub * 8) = o;
+  *reinterpret_cast<uint4*>(p.dq + (tok0 + i) * p.rs_dq + h * D + sub * 8) = o;
 }
 
 template <int D>
@@ -169,13 +209,6 @@ struct BwdLayout {
 #endif
 constexpr int kPolyPairsBwd = FA_BWD_POLY_PAIRS;
 
-enum : unsigned int {
-  kSiteBwdProducer = 0x201,
-  kSiteBwdMma = 0x202,
-  kSiteBwdSoftmax = 0x203,
-  kSiteBwdDrain = 0x204,
-  kSiteBwdSmemAlign = 0x2FF
-};
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -209,7 +242,9 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
 // Trace slot of (role, iteration, event) for the traced CTA (block 0).
 #define FA_BWD_TR(role, n, e) ((((role) * 128 + ((n) & 127)) * 8) + (e))
 
-template <int D, bool CAUSAL>
+// GENERAL = false compiles the plain dense case (no sequence offsets, no window,
+// CAUSAL fixed); GENERAL = true reads the window and cu_seqlens at run time.
+template <int D, bool CAUSAL, bool GENERAL>
 __global__ void __launch_bounds__(448, 1)
     bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -229,7 +264,6 @@ __global__ void __launch_bounds__(448, 1)
 #define BAR(i) (bar0 + 8u * static_cast<uint32_t>(i))
 
   const int warp = warp_id(), lane = lane_id();
-  const int BH = p.B * p.H;
   // Heads in groups of head_group (L2 reuse of Q/dO and the dQ accumulator); within a
   // group, key tile 0 (the most query tiles when causal) first.
   const int G = p.head_group;
@@ -239,8 +273,22 @@ __global__ void __launch_bounds__(448, 1)
   const int jt = rem / G;
   const int bh = grp * G + rem % G;
   const int b = bh / p.H, h = bh % p.H;
-  const int it0 = CAUSAL ? jt : 0;
-  const int niter = p.nqt - it0;
+  long long tok0 = static_cast<long long>(b) * p.N;  // first token of the sequence
+  int seqlen = p.N;
+  if (GENERAL && !bwd_seq(p, b, &tok0, &seqlen)) return;  // reported by the preprocessing kernel
+  const bool var = GENERAL && p.cu_seqlens != nullptr;
+  const int tb = var ? 0 : b;                            // batch coordinate of the maps
+  const int trow = var ? static_cast<int>(tok0) : 0;     // row coordinate of row 0
+  if (jt * 128 >= seqlen) return;  // key tile past the end of a shorter sequence
+  // Query tiles [it0, it0 + niter) see at least one key of this tile: keys
+  // [k0, k1] are visible to queries [k0 - wr, k1 + wl] within [0, L).
+  const int wl = GENERAL ? p.window_left : -1;
+  const int wr = GENERAL ? p.window_right : (CAUSAL ? 0 : -1);
+  const int k0 = jt * 128, k1 = min(seqlen, k0 + 128) - 1;
+  const int qlo = wr < 0 ? 0 : max(0, k0 - wr);
+  const int qhi = wl < 0 ? seqlen - 1 : min(seqlen - 1, k1 + wl);
+  const int it0 = qlo / 128;
+  const int niter = qhi / 128 - it0 + 1;  // >= 1: every key sees at least itself
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(L::kKVFull), 1);
@@ -282,8 +330,8 @@ __global__ void __launch_bounds__(448, 1)
       tma_prefetch_desc(&tmdO);
       mbar_arrive_expect_tx(BAR(L::kKVFull), 2 * L::kTile);
       for (int bx = 0; bx < D / 64; ++bx) {
-        tma_load_4d(sK + bx * 16384, &tmK, BAR(L::kKVFull), bx * 64, h, jt * 128, b);
-        tma_load_4d(sV + bx * 16384, &tmV, BAR(L::kKVFull), bx * 64, h, jt * 128, b);
+        tma_load_4d(sK + bx * 16384, &tmK, BAR(L::kKVFull), bx * 64, h, trow + jt * 128, tb);
+        tma_load_4d(sV + bx * 16384, &tmV, BAR(L::kKVFull), bx * 64, h, trow + jt * 128, tb);
       }
       const float* lse2_h = p.lse2 + static_cast<size_t>(bh) * p.Np;
       const float* dvec_h = p.dvec + static_cast<size_t>(bh) * p.Np;
@@ -297,7 +345,7 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t sQ = base + L::kQ0 + s * L::kTile;
         mbar_arrive_expect_tx(BAR(L::kQFull + s), L::kTile + 1024);
         for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_4d(sQ + bx * 16384, &tmQ, BAR(L::kQFull + s), bx * 64, h, it * 128, b);
+          tma_load_4d(sQ + bx * 16384, &tmQ, BAR(L::kQFull + s), bx * 64, h, trow + it * 128, tb);
         const uint32_t sv = base + L::kVec + s * 1024;
         bulk_load(sv, lse2_h + it * 128, 512, BAR(L::kQFull + s));
         bulk_load(sv + 512, dvec_h + it * 128, 512, BAR(L::kQFull + s));
@@ -306,7 +354,7 @@ __global__ void __launch_bounds__(448, 1)
         FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(3, n, 1));
         mbar_arrive_expect_tx(BAR(L::kDOFull), L::kTile);
         for (int bx = 0; bx < D / 64; ++bx)
-          tma_load_4d(base + L::kDO + bx * 16384, &tmdO, BAR(L::kDOFull), bx * 64, h, it * 128, b);
+          tma_load_4d(base + L::kDO + bx * 16384, &tmdO, BAR(L::kDOFull), bx * 64, h, trow + it * 128, tb);
         ++ndo;
       }
       // Never leave the CTA with copies in flight.
@@ -424,7 +472,7 @@ __global__ void __launch_bounds__(448, 1)
     const int c0 = half * 64;  // first query column of this warpgroup
     const int r = wq * 32 + lane;
     const int key = jt * 128 + r;
-    const bool key_ok = key < p.N;
+    const bool key_ok = key < seqlen;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float sl2 = p.scale_log2;
     const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
@@ -446,8 +494,12 @@ __global__ void __launch_bounds__(448, 1)
       reg_fence32(s0);
       reg_fence32(s1);
       FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 1));
-      // Local columns c < qlim are not visible to this key: query < key (causal) or key >= N.
-      const int qlim = !key_ok ? 1 << 30 : (CAUSAL ? key - it * 128 - c0 : 0);
+      // Local columns c in [qlo_c, qhi_c] are the queries that see this key (window
+      // [key - wr, key + wl]); none if the key is past the sequence. Queries past the
+      // sequence have lse2 = +inf, so their P is already 0.
+      const int q0 = it * 128 + c0;
+      const int qlo_c = !key_ok ? (1 << 30) : (wr < 0 ? -(1 << 30) : key - wr - q0);
+      const int qhi_c = wl < 0 ? (1 << 30) : key + wl - q0;
       uint32_t pk[32];
 #pragma unroll
       for (int c2 = 0; c2 < 32; ++c2) {
@@ -461,8 +513,8 @@ __global__ void __launch_bounds__(448, 1)
           e0 = ex2_approx(e0);  // MUFU
           e1 = ex2_approx(e1);
         }
-        const float p0 = (c < qlim) ? 0.f : e0;
-        const float p1 = (c + 1 < qlim) ? 0.f : e1;
+        const float p0 = (c < qlo_c || c > qhi_c) ? 0.f : e0;
+        const float p1 = (c + 1 < qlo_c || c + 1 > qhi_c) ? 0.f : e1;
         pk[c2] = pack_bf16x2(p0, p1);
       }
       tmem_st32(tS + lane_off + c0 / 2, pk);  // P^T bf16: two queries per 32-bit column
@@ -515,10 +567,9 @@ __global__ void __launch_bounds__(448, 1)
     if (ok) {
       // Epilogue: warpgroup 0 writes dV rows, warpgroup 1 writes dK rows (x scale).
       tc_fence_after();
-      const size_t orow = ((static_cast<size_t>(b) * p.N + key) * p.H + h) * D;
       const uint32_t tsrc = (half == 0 ? tDV : tDK) + lane_off;
       const float mul = half == 0 ? 1.f : p.scale;
-      uint16_t* dst = (half == 0 ? p.dv : p.dk) + orow;
+      uint16_t* dst = (half == 0 ? p.dv + (tok0 + key) * p.rs_dv : p.dk + (tok0 + key) * p.rs_dk) + h * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -599,7 +650,7 @@ __global__ void __launch_bounds__(448, 1)
           tmem_ld32(tDQ + lane_off + cc * 32, o);
           tmem_wait_ld();
           reg_fence32(o);
-          if (qrow < p.N) {
+          if (qrow < seqlen) {
 #pragma unroll
             for (int v = 0; v < 8; ++v)
               red_add_v4(dst + cc * 32 + 4 * v, __uint_as_float(o[4 * v]) * sc,

@@ -123,17 +123,29 @@ fa_status get_encoder(EncodeTiledFn* fn) {
   return FA_OK;
 }
 
-// 4-D map over a [B, N, H, d] bf16 tensor; one box = 128 rows of one (b, h) x 64
-// columns of d, stored with the 128-byte swizzle the UMMA descriptors expect.
-fa_status map_bnhd(CUtensorMap* map, const void* ptr, int B, int N, int H, int d) {
+// Row layout shared by every [*, H, d] bf16 operand of one call: dense batches of N
+// rows (row (b, n) is token b*N + n) or one packed batch of `total` tokens split into
+// sequences by cu_seqlens. Consecutive tokens of an operand are `rs` elements apart.
+struct RowLayout {
+  int B, N, H, d;
+  const int* cu_seqlens;  // NULL: dense
+  int total;              // variable length only
+};
+
+// 4-D map over one operand; one box = 128 rows of one head x 64 columns of d, stored
+// with the 128-byte swizzle the UMMA descriptors expect. Dense: dims (d, H, N, B) with
+// row coordinate n and batch coordinate b. Variable length: dims (d, H, total, 1) with
+// row coordinate = token.
+fa_status map_rows(CUtensorMap* map, const void* ptr, const RowLayout& lay, long long rs) {
   EncodeTiledFn enc;
   fa_status st = get_encoder(&enc);
   if (st != FA_OK) return st;
-  const cuuint64_t gdim[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(H),
-                              static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(B)};
-  const cuuint64_t gstride[3] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(H) * d * 2,
-                                 static_cast<cuuint64_t>(N) * H * d * 2};
+  const bool var = lay.cu_seqlens != nullptr;
+  const cuuint64_t rows = static_cast<cuuint64_t>(var ? lay.total : lay.N);
+  const cuuint64_t gdim[4] = {static_cast<cuuint64_t>(lay.d), static_cast<cuuint64_t>(lay.H), rows,
+                              static_cast<cuuint64_t>(var ? 1 : lay.B)};
+  const cuuint64_t gstride[3] = {static_cast<cuuint64_t>(lay.d) * 2, static_cast<cuuint64_t>(rs) * 2,
+                                 rows * static_cast<cuuint64_t>(rs) * 2};
   const cuuint32_t box[4] = {64, 1, 128, 1};
   const cuuint32_t estride[4] = {1, 1, 1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), gdim, gstride,
@@ -165,11 +177,11 @@ fa_status check_launch(const char* what) {
   return FA_OK;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool GENERAL>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const fa::FwdParams& p, int dev, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
-  auto kern = fa::fwd_kernel<D, CAUSAL>;
+  auto kern = fa::fwd_kernel<D, CAUSAL, GENERAL>;
   fa_status st = set_smem(kern, L::kAlloc, dev);
   if (st != FA_OK) return st;
   const unsigned grid = static_cast<unsigned>(p.num_qblocks) * p.B * p.H;
@@ -178,11 +190,11 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 }
 
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool GENERAL>
 fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                           const CUtensorMap& mdo, const fa::BwdParams& p, int dev, cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
-  auto kern = fa::bwd_kernel<D, CAUSAL>;
+  auto kern = fa::bwd_kernel<D, CAUSAL, GENERAL>;
   fa_status st = set_smem(kern, L::kBytes, dev);
   if (st != FA_OK) return st;
   const unsigned grid = static_cast<unsigned>(p.nqt) * p.B * p.H;
@@ -190,16 +202,24 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   return check_launch("fa_bwd main kernel launch");
 }
 
+// Strides (elements between consecutive tokens) of the eight row-major operands of a
+// backward call, in the order q, k, v, out, dout, dq, dk, dv.
+struct BwdStrides {
+  long long q, k, v, o, dout, dq, dk, dv;
+};
+
 fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
-                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
-                  bool causal, float scale, void* workspace, const fa::BwdWorkspace& ws, int dev,
-                  cudaStream_t stream, cudaEvent_t ev_start, cudaEvent_t ev_stop) {
+                  const float* lse, void* dq, void* dk, void* dv, const RowLayout& lay,
+                  const BwdStrides& rs, int wl, int wr, float scale, void* workspace,
+                  const fa::BwdWorkspace& ws, int dev, cudaStream_t stream, cudaEvent_t ev_start,
+                  cudaEvent_t ev_stop) {
+  const int B = lay.B, H = lay.H, N = lay.N, d = lay.d;
   CUtensorMap mq, mk, mv, mdo;
   fa_status st;
-  if ((st = map_bnhd(&mq, q, B, N, H, d)) != FA_OK) return st;
-  if ((st = map_bnhd(&mk, k, B, N, H, d)) != FA_OK) return st;
-  if ((st = map_bnhd(&mv, v, B, N, H, d)) != FA_OK) return st;
-  if ((st = map_bnhd(&mdo, dout, B, N, H, d)) != FA_OK) return st;
+  if ((st = map_rows(&mq, q, lay, rs.q)) != FA_OK) return st;
+  if ((st = map_rows(&mk, k, lay, rs.k)) != FA_OK) return st;
+  if ((st = map_rows(&mv, v, lay, rs.v)) != FA_OK) return st;
+  if ((st = map_rows(&mdo, dout, lay, rs.dout)) != FA_OK) return st;
   fa::BwdParams p;
   p.B = B;
   p.H = H;
@@ -208,8 +228,17 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   p.nqt = p.Np / 128;
   // Four heads: their Q, dO and fp32 dQ accumulator (4 x 16 MiB at N = 16384) fit in L2.
   p.head_group = head_group_for(B * H, 4);
+  p.window_left = wl;
+  p.window_right = wr;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.cu_seqlens = lay.cu_seqlens;
+  p.total = lay.total;
+  p.rs_o = rs.o;
+  p.rs_do = rs.dout;
+  p.rs_dq = rs.dq;
+  p.rs_dk = rs.dk;
+  p.rs_dv = rs.dv;
   p.out = static_cast<const uint16_t*>(out);
   p.dout = static_cast<const uint16_t*>(dout);
   p.lse = lse;
@@ -229,10 +258,15 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   cudaError_t e;
   if (ev_start && (e = cudaEventRecord(ev_start, stream)) != cudaSuccess)
     return cuda_fail(e, "fa_bwd_profiled: record start event");
-  if (d == 64) st = causal ? launch_bwd_main<64, true>(mq, mk, mv, mdo, p, dev, stream)
-                           : launch_bwd_main<64, false>(mq, mk, mv, mdo, p, dev, stream);
-  else st = causal ? launch_bwd_main<128, true>(mq, mk, mv, mdo, p, dev, stream)
-                   : launch_bwd_main<128, false>(mq, mk, mv, mdo, p, dev, stream);
+  const bool general = lay.cu_seqlens != nullptr || wl >= 0 || wr > 0;
+  if (d == 64)
+    st = general ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, dev, stream)
+         : wr == 0 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, dev, stream)
+                   : launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, dev, stream);
+  else
+    st = general ? launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, dev, stream)
+         : wr == 0 ? launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, dev, stream)
+                   : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, dev, stream);
   if (st != FA_OK) return st;
   if (ev_stop && (e = cudaEventRecord(ev_stop, stream)) != cudaSuccess)
     return cuda_fail(e, "fa_bwd_profiled: record stop event");
@@ -241,6 +275,78 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   if (d == 64) fa::bwd_dq_convert_kernel<64><<<cv_blocks, 256, 0, stream>>>(p);
   else fa::bwd_dq_convert_kernel<128><<<cv_blocks, 256, 0, stream>>>(p);
   return check_launch("fa_bwd dq convert launch");
+}
+
+fa_status run_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
+                  const RowLayout& lay, long long rs_q, long long rs_k, long long rs_v,
+                  long long rs_o, int wl, int wr, float scale, int dev, cudaStream_t stream) {
+  CUtensorMap mq, mk, mv;
+  fa_status st;
+  if ((st = map_rows(&mq, q, lay, rs_q)) != FA_OK) return st;
+  if ((st = map_rows(&mk, k, lay, rs_k)) != FA_OK) return st;
+  if ((st = map_rows(&mv, v, lay, rs_v)) != FA_OK) return st;
+  fa::FwdParams p;
+  p.B = lay.B;
+  p.H = lay.H;
+  p.N = lay.N;
+  p.num_qblocks = (lay.N + 255) / 256;
+  // Eight heads: their K and V (8 x 4 MiB at N = 8192) stay in L2 while their CTAs run.
+  p.head_group = head_group_for(lay.B * lay.H, 8);
+  p.window_left = wl;
+  p.window_right = wr;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.cu_seqlens = lay.cu_seqlens;
+  p.total = lay.total;
+  p.o_rs = rs_o;
+  p.out = static_cast<uint16_t*>(out);
+  p.lse = lse;
+  // Plain dense problems (no sequence offsets, no window beyond causal) take the
+  // kernel instance with those tests compiled out.
+  const bool general = lay.cu_seqlens != nullptr || wl >= 0 || wr > 0;
+  if (lay.d == 64) {
+    if (general) return launch_fwd<64, false, true>(mq, mk, mv, p, dev, stream);
+    return wr == 0 ? launch_fwd<64, true, false>(mq, mk, mv, p, dev, stream)
+                   : launch_fwd<64, false, false>(mq, mk, mv, p, dev, stream);
+  }
+  if (general) return launch_fwd<128, false, true>(mq, mk, mv, p, dev, stream);
+  return wr == 0 ? launch_fwd<128, true, false>(mq, mk, mv, p, dev, stream)
+                 : launch_fwd<128, false, false>(mq, mk, mv, p, dev, stream);
+}
+
+// Checks shared by the extended entry points; on success fills `lay`, `wr_eff` (the
+// right window edge with causal folded in) and returns FA_OK. `*empty` is set when the
+// call has no work.
+fa_status check_ex(const char* who, const int* cu_seqlens, int total_tokens, int B, int H, int N,
+                   int d, int causal, int window_left, int window_right, float scale,
+                   const long long* strides, int nstrides, RowLayout* lay, int* wr_eff, bool* empty) {
+  if (B < 0 || H < 0 || N < 0 || total_tokens < 0)
+    return fail(FA_ERR_INVALID_ARG, "%s: negative size B=%d H=%d N=%d total=%d", who, B, H, N, total_tokens);
+  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "%s: head dim %d not supported (64 or 128)", who, d);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "%s: scale must be finite", who);
+  if (window_left < -1 || window_right < -1)
+    return fail(FA_ERR_INVALID_ARG, "%s: window edges must be >= 0, or -1 for unbounded", who);
+  if (causal && window_right > 0)
+    return fail(FA_ERR_INVALID_ARG, "%s: causal attention needs window_right 0 or -1 (got %d)", who,
+                window_right);
+  for (int i = 0; i < nstrides; ++i)
+    if (strides[i] < static_cast<long long>(H) * d || strides[i] % 8 != 0)
+      return fail(FA_ERR_INVALID_ARG,
+                  "%s: row stride %lld must be a multiple of 8 elements and at least H*d = %d", who,
+                  strides[i], H * d);
+  const long long nkb = (static_cast<long long>(N) + 127) / 128;  // backward grid per (b, h)
+  if (nkb * B * H >= (1LL << 31) || N > (1 << 30) || H > (1 << 20))
+    return fail(FA_ERR_INVALID_ARG, "%s: problem too large (B=%d H=%d N=%d)", who, B, H, N);
+  lay->B = B;
+  lay->N = N;
+  lay->H = H;
+  lay->d = d;
+  lay->cu_seqlens = cu_seqlens;
+  lay->total = cu_seqlens ? total_tokens : 0;
+  *wr_eff = causal ? 0 : window_right;
+  *empty = B == 0 || H == 0 || N == 0 || (cu_seqlens && total_tokens == 0);
+  if (cu_seqlens && !aligned4(cu_seqlens))
+    return fail(FA_ERR_INVALID_ARG, "%s: cu_seqlens must be 4-byte aligned", who);
+  return FA_OK;
 }
 
 // CTAs per (batch, head) for decode: a power of two <= 8 (one portable cluster)
@@ -330,25 +436,31 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   int dev = 0;
   fa_status st = current_device(&dev, nullptr);
   if (st != FA_OK) return st;
-  CUtensorMap mq, mk, mv;
-  if ((st = map_bnhd(&mq, q, B, N, H, d)) != FA_OK) return st;
-  if ((st = map_bnhd(&mk, k, B, N, H, d)) != FA_OK) return st;
-  if ((st = map_bnhd(&mv, v, B, N, H, d)) != FA_OK) return st;
-  fa::FwdParams p;
-  p.B = B;
-  p.H = H;
-  p.N = N;
-  p.num_qblocks = static_cast<int>(nqb);
-  // Eight heads: their K and V (8 x 4 MiB at N = 8192) stay in L2 while their CTAs run.
-  p.head_group = head_group_for(B * H, 8);
-  p.nkv_total = (N + 127) / 128;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.out = static_cast<uint16_t*>(out);
-  p.lse = lse;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d == 64)
-    return causal ? launch_fwd<64, true>(mq, mk, mv, p, dev, s) : launch_fwd<64, false>(mq, mk, mv, p, dev, s);
-  return causal ? launch_fwd<128, true>(mq, mk, mv, p, dev, s) : launch_fwd<128, false>(mq, mk, mv, p, dev, s);
+  const RowLayout lay{B, N, H, d, nullptr, 0};
+  const long long rs = static_cast<long long>(H) * d;
+  return run_fwd(q, k, v, out, lse, lay, rs, rs, rs, rs, -1, causal ? 0 : -1, scale, dev,
+                 static_cast<cudaStream_t>(stream));
+}
+
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                    const int* cu_seqlens, int total_tokens, int B, int H, int N, int d,
+                    long long q_row_stride, long long k_row_stride, long long v_row_stride,
+                    long long out_row_stride, int causal, int window_left, int window_right,
+                    float scale, void* stream) {
+  const long long strides[4] = {q_row_stride, k_row_stride, v_row_stride, out_row_stride};
+  RowLayout lay;
+  int wr = -1;
+  bool empty = false;
+  fa_status st = check_ex("fa_fwd_ex", cu_seqlens, total_tokens, B, H, N, d, causal, window_left,
+                          window_right, scale, strides, 4, &lay, &wr, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd_ex: null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_fwd_ex: q/k/v/out must be 16-byte aligned, lse 4-byte aligned");
+  int dev = 0;
+  if ((st = current_device(&dev, nullptr)) != FA_OK) return st;
+  return run_fwd(q, k, v, out, lse, lay, q_row_stride, k_row_stride, v_row_stride, out_row_stride,
+                 window_left, wr, scale, dev, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
@@ -381,9 +493,42 @@ fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const voi
   int dev = 0;
   fa_status st = current_device(&dev, nullptr);
   if (st != FA_OK) return st;
-  return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, N, d, causal != 0, scale, workspace, ws,
-                 dev, static_cast<cudaStream_t>(stream),
+  const RowLayout lay{B, N, H, d, nullptr, 0};
+  const long long rs = static_cast<long long>(H) * d;
+  const BwdStrides strides{rs, rs, rs, rs, rs, rs, rs, rs};
+  return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, lay, strides, -1, causal ? 0 : -1, scale,
+                 workspace, ws, dev, static_cast<cudaStream_t>(stream),
                  static_cast<cudaEvent_t>(main_start), static_cast<cudaEvent_t>(main_stop));
+}
+
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens,
+                    int total_tokens, int B, int H, int N, int d, const long long* row_strides,
+                    int causal, int window_left, int window_right, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  if (!row_strides) return fail(FA_ERR_INVALID_ARG, "fa_bwd_ex: row_strides is null");
+  RowLayout lay;
+  int wr = -1;
+  bool empty = false;
+  fa_status st = check_ex("fa_bwd_ex", cu_seqlens, total_tokens, B, H, N, d, causal, window_left,
+                          window_right, scale, row_strides, 8, &lay, &wr, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !out || !dout || !lse || !dq || !dk || !dv)
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd_ex: null pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned16(dout) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv) || !aligned4(lse))
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd_ex: tensors must be 16-byte aligned, lse 4-byte aligned");
+  const fa::BwdWorkspace ws = fa::bwd_ws_layout(B, H, N, d);
+  if (!workspace || workspace_bytes < ws.total)
+    return fail(FA_ERR_WORKSPACE, "fa_bwd_ex: workspace needs %zu bytes, got %zu", ws.total, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(FA_ERR_INVALID_ARG, "fa_bwd_ex: workspace must be 256-byte aligned");
+  int dev = 0;
+  if ((st = current_device(&dev, nullptr)) != FA_OK) return st;
+  const BwdStrides strides{row_strides[0], row_strides[1], row_strides[2], row_strides[3],
+                           row_strides[4], row_strides[5], row_strides[6], row_strides[7]};
+  return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, lay, strides, window_left, wr, scale, workspace,
+                 ws, dev, static_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,

@@ -34,13 +34,17 @@
 namespace fa {
 
 struct FwdParams {
-  int B, H, N;
-  int num_qblocks;   // ceil(N / 256): CTAs per (batch, head)
-  int head_group;    // heads scheduled together (divides B*H), for L2 reuse of K/V
-  int nkv_total;     // ceil(N / 128): key tiles per head
-  float scale_log2;  // scale * log2(e)
-  uint16_t* out;     // [B, N, H, d] bf16
-  float* lse;        // [B, H, N] fp32, natural log
+  int B, H, N;        // N: sequence length (dense) or the largest one (variable length)
+  int num_qblocks;    // ceil(N / 256): CTAs per (batch, head)
+  int head_group;     // heads scheduled together (divides B*H), for L2 reuse of K/V
+  int window_left;    // keys visible to query i: [i - window_left, i + window_right];
+  int window_right;   // -1 = unbounded on that side (causal: window_right = 0)
+  float scale_log2;   // scale * log2(e)
+  const int* cu_seqlens;  // NULL: dense [B, N] rows; else [B + 1] token offsets
+  int total;          // variable length: tokens in the packed tensors
+  long long o_rs;     // elements between consecutive rows (tokens) of out
+  uint16_t* out;      // dense: row (b, n) at (b*N + n)*o_rs; variable: token t at t*o_rs
+  float* lse;         // dense [B, H, N]; variable [H, total]; fp32, natural log
 };
 
 // The softmax of a 128-row tile is split over kFwdGroups groups of four warps, each
@@ -109,7 +113,12 @@ constexpr bool kAluPack = FA_FWD_ALU_PACK != 0;
 constexpr int kL2Prefetch = FA_FWD_L2_PREFETCH;
 
 // Site ids for timeout reports.
-enum : unsigned int { kSiteFwdProducer = 0x101, kSiteFwdMma = 0x102, kSiteFwdSoftmax = 0x103 };
+enum : unsigned int {
+  kSiteFwdProducer = 0x101,
+  kSiteFwdMma = 0x102,
+  kSiteFwdSoftmax = 0x103,
+  kSiteFwdSeqlens = 0x104
+};
 
 // Max / min of 128 values held as two 64-element halves, with 8 independent
 // accumulators so the reduction is 10 dependent steps deep instead of 64.
@@ -137,7 +146,10 @@ __device__ __forceinline__ float row_min128(const float (&x)[64], const float (&
 // Trace slot of (role, key tile, event) for the traced CTA (block 0).
 #define FA_FWD_TR(role, j, e) ((((role) * 128 + ((j) & 127)) * 16) + (e))
 
-template <int D, bool CAUSAL>
+// GENERAL = false compiles the plain dense case (no sequence offsets, no window,
+// CAUSAL fixed) with every window and varlen test folded away; GENERAL = true reads
+// the window and cu_seqlens from the parameters (CAUSAL is then unused).
+template <int D, bool CAUSAL, bool GENERAL>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -166,14 +178,39 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const int bh = grp * G + rem % G;
   const int b = bh / p.H;
   const int h = bh % p.H;
-  int row0[2], nkv[2];
+  // Sequence of this CTA: its first token (TMA row coordinate and batch coordinate)
+  // and its length L. Dense tensors are indexed (row, b); variable-length ones are a
+  // single batch of tokens indexed (cu_seqlens[b] + row, 0).
+  int seq0 = 0, seqlen = p.N, tb = b;
+  if (GENERAL && p.cu_seqlens != nullptr) {
+    const int s0 = __ldg(p.cu_seqlens + b), s1 = __ldg(p.cu_seqlens + b + 1);
+    seq0 = s0;
+    seqlen = s1 - s0;
+    tb = 0;
+    if (s0 < 0 || seqlen < 0 || seqlen > p.N || s1 > p.total) {
+      if (threadIdx.x == 0 && qb == 0 && h == 0) report(kDevBadInput, kSiteFwdSeqlens, b);
+      return;  // uniform over the CTA, before any barrier or TMEM allocation
+    }
+  }
+  const int wl = GENERAL ? p.window_left : -1;
+  const int wr = GENERAL ? p.window_right : (CAUSAL ? 0 : -1);
+  // Key tiles [ka[t], kb[t]] reach at least one row of Q tile t: rows [r, r + 128)
+  // see keys [r - wl, r + 127 + wr] within [0, L).
+  int row0[2], ka[2], kb[2], nkv[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     row0[t] = qb * 256 + t * 128;
-    const bool valid = row0[t] < p.N;
-    nkv[t] = !valid ? 0 : (CAUSAL ? min(row0[t] / 128 + 1, p.nkv_total) : p.nkv_total);
+    const int lo = wl < 0 ? 0 : max(0, row0[t] - wl);
+    const int hi = wr < 0 ? seqlen - 1 : min(seqlen - 1, row0[t] + 127 + wr);
+    ka[t] = lo / 128;
+    kb[t] = hi < 0 ? -1 : hi / 128;
+    nkv[t] = (row0[t] < seqlen && lo <= hi) ? kb[t] - ka[t] + 1 : 0;
   }
-  const int nkv_max = max(nkv[0], nkv[1]);
+  // Key tiles the CTA streams: [J0, J0 + nkv_max).
+  const int J0 = nkv[0] > 0 ? (nkv[1] > 0 ? min(ka[0], ka[1]) : ka[0]) : ka[1];
+  const int J1 = nkv[1] > 0 ? (nkv[0] > 0 ? max(kb[0], kb[1]) : kb[1]) : kb[0];
+  const int nkv_max = (nkv[0] > 0 || nkv[1] > 0) ? J1 - J0 + 1 : 0;
+  if (nkv_max == 0) return;  // rows past the end of a shorter sequence
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -213,20 +250,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_arrive_expect_tx(BAR(L::kQFull + t), L::kTileBytes);
         for (int bx = 0; bx < D / 64; ++bx)
           tma_load_4d(sQ + t * L::kTileBytes + bx * 16384, &tmQ, BAR(L::kQFull + t), bx * 64, h,
-                      row0[t], b);
+                      seq0 + row0[t], tb);
       }
       int it = 0;
       if (kL2Prefetch > 0)
         for (int j = 0; j < kL2Prefetch && j < nkv_max; ++j)
           for (int kv = 0; kv < 2; ++kv)
             for (int bx = 0; bx < D / 64; ++bx)
-              tma_prefetch_l2_4d(kv ? &tmV : &tmK, bx * 64, h, j * 128, b);
+              tma_prefetch_l2_4d(kv ? &tmV : &tmK, bx * 64, h, seq0 + (J0 + j) * 128, tb);
       for (int j = 0; j < nkv_max; ++j) {
         bool stop = false;
         if (kL2Prefetch > 0 && j + kL2Prefetch < nkv_max)
           for (int kv = 0; kv < 2; ++kv)
             for (int bx = 0; bx < D / 64; ++bx)
-              tma_prefetch_l2_4d(kv ? &tmV : &tmK, bx * 64, h, (j + kL2Prefetch) * 128, b);
+              tma_prefetch_l2_4d(kv ? &tmV : &tmK, bx * 64, h, seq0 + (J0 + j + kL2Prefetch) * 128, tb);
         for (int kv = 0; kv < 2; ++kv) {
           const int s = it % L::kStages;
           const uint32_t ph = (it / L::kStages) & 1;
@@ -239,7 +276,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const CUtensorMap* m = kv ? &tmV : &tmK;
           for (int bx = 0; bx < D / 64; ++bx)
             tma_load_4d(sKV + s * L::kTileBytes + bx * 16384, m, BAR(L::kKVFull + s), bx * 64, h,
-                        j * 128, b);
+                        seq0 + (J0 + j) * 128, tb);
           ++it;
         }
         if (stop) break;
@@ -288,37 +325,53 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           umma_ts_w(tO, tS + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
         }
       };
+      // Ring item x is K (x even) or V (x odd) of key tile J0 + x / 2. This tile reads
+      // key tiles J0 + a .. J0 + a + n - 1: items 2a .. 2(a + n) - 1.
       const int n = nkv[t];
-      if (n > 0) {
+      const int a = n > 0 ? ka[t] - J0 : nkv_max;
+      // Releases ring items [from, to) that this tile does not read.
+      auto skip_items = [&](int from, int to) {
+        for (int x = from; x < to && ok; ++x) {
+          const int s = x % L::kStages;
+          ok = __all_sync(0xffffffffu,
+                          wait_bar(BAR(L::kKVFull + s), (x / L::kStages) & 1, abort_flag, kSiteFwdMma));
+          if (ok && lane == 0) mbar_arrive(BAR(L::kKVEmpty + s));
+        }
+      };
+      skip_items(0, 2 * a);
+      if (n > 0 && ok) {
+        const int ik0 = 2 * a, sk0 = ik0 % L::kStages;
         ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kQFull + t), 0, abort_flag, kSiteFwdMma) &&
-                                         wait_bar(BAR(L::kKVFull + 0), 0, abort_flag, kSiteFwdMma));
+                                         wait_bar(BAR(L::kKVFull + sk0), (ik0 / L::kStages) & 1,
+                                                  abort_flag, kSiteFwdMma));
         if (ok) {
           tc_fence_after();
-          issue_qk(0);
+          issue_qk(sk0);
           umma_commit_w(BAR(L::kSFull + t));
-          umma_commit_w(BAR(L::kKVEmpty + 0));
+          umma_commit_w(BAR(L::kKVEmpty + sk0));
         }
       }
-      for (int j = 0; j < n && ok; ++j) {
-        const int iv = 2 * j + 1, ik = 2 * j + 2;
+      for (int i = 0; i < n && ok; ++i) {  // i-th key tile of this Q tile
+        const int jr = a + i;
+        const int iv = 2 * jr + 1, ik = 2 * jr + 2;
         const int sv = iv % L::kStages, sk = ik % L::kStages;
         ok = __all_sync(0xffffffffu,
                         wait_bar(BAR(L::kKVFull + sv), (iv / L::kStages) & 1, abort_flag, kSiteFwdMma));
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 10 * t));
-        if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kPHalf + 2 * t + 0), j & 1, abort_flag, kSiteFwdMma));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, jr, 10 * t));
+        if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kPHalf + 2 * t + 0), i & 1, abort_flag, kSiteFwdMma));
         if (!ok) break;
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 1 + 4 * t));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, jr, 1 + 4 * t));
         tc_fence_after();
-        issue_pv_half(sv, 0, j > 0);
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 2 + 4 * t));
-        if (!__all_sync(0xffffffffu, wait_bar(BAR(L::kPHalf + 2 * t + 1), j & 1, abort_flag, kSiteFwdMma))) {
+        issue_pv_half(sv, 0, i > 0);
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, jr, 2 + 4 * t));
+        if (!__all_sync(0xffffffffu, wait_bar(BAR(L::kPHalf + 2 * t + 1), i & 1, abort_flag, kSiteFwdMma))) {
           ok = false;
           break;
         }
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 3 + 4 * t));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, jr, 3 + 4 * t));
         tc_fence_after();
-        issue_pv_half(sv, 1, j > 0);
-        const bool more = j + 1 < n;
+        issue_pv_half(sv, 1, i > 0);
+        const bool more = i + 1 < n;
         if (more) {
           if (!__all_sync(0xffffffffu,
                           wait_bar(BAR(L::kKVFull + sk), (ik / L::kStages) & 1, abort_flag, kSiteFwdMma))) {
@@ -333,14 +386,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         umma_commit_w(BAR(L::kKVEmpty + sv));
         if (more) umma_commit_w(BAR(L::kKVEmpty + sk));
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, j, 4 + 4 * t));
+        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_FWD_TR(0, jr, 4 + 4 * t));
       }
-      // Ring loads after this tile's last key tile: K_n, V_n, ..., V_(nkv_max - 1).
-      for (int x = 2 * n; x < 2 * nkv_max && ok; ++x) {
-        const int s = x % L::kStages;
-        ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kKVFull + s), (x / L::kStages) & 1, abort_flag, kSiteFwdMma));
-        if (ok && lane == 0) mbar_arrive(BAR(L::kKVEmpty + s));
-      }
+      // Ring loads after this tile's last key tile.
+      skip_items(n > 0 ? 2 * (a + n) : 2 * nkv_max, 2 * nkv_max);
       // Let every issued MMA finish before TMEM can be released.
       umma_commit_w(BAR(L::kDrain + t));
       drain_wait(BAR(L::kDrain + t), 0);
@@ -369,15 +418,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float m[2] = {-INFINITY, -INFINITY};  // running row max per tile (log2 units)
     float l[2] = {0.f, 0.f};              // running exp-sum over this group's columns
     bool ok = true;
-    for (int j = 0; j < nkv_max && ok; ++j) {
+    for (int jr = 0; jr < nkv_max && ok; ++jr) {
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
-        if (j >= nkv[t]) continue;  // uniform over the CTA
+        const int i = jr - (ka[t] - J0);  // step index within this Q tile's key tiles
+        if (i < 0 || i >= nkv[t]) continue;  // uniform over the CTA
+        const int j = J0 + jr;               // key tile
         const int row_g = row0[t] + r;
         const uint32_t tS = tmem + t * 128 + lane_off;
         const uint32_t tO = tmem + 256 + t * D + lane_off;
         const bool w_ok = __all_sync(0xffffffffu,
-                                     wait_bar(BAR(L::kSFull + t), j & 1, abort_flag, kSiteFwdSoftmax));
+                                     wait_bar(BAR(L::kSFull + t), i & 1, abort_flag, kSiteFwdSoftmax));
         FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 0));
         tc_fence_after();
         float x[C];
@@ -394,12 +445,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 1));
         const int kbase = j * 128 + C * grp;  // key index of this group's column 0
-        const bool masked = (CAUSAL && j * 128 == row0[t]) || (j * 128 + 128 > p.N);
+        // A tile needs per-element masking if it reaches past the sequence or outside
+        // the window of some row of the Q tile (causal: the diagonal tile).
+        const int k0 = j * 128;
+        const bool masked = (k0 + 128 > seqlen) || (wl >= 0 && k0 < row0[t] + 127 - wl) ||
+                            (wr >= 0 && k0 + 127 > row0[t] + wr);
         if (masked) {
           // Diagonal or tail tile: scale first, then mask to -inf.
-          const int lim = CAUSAL ? min(row_g, p.N - 1) : p.N - 1;
+          const int lim = wr < 0 ? seqlen - 1 : min(row_g + wr, seqlen - 1);
+          const int first = wl < 0 ? 0 : row_g - wl;
 #pragma unroll
-          for (int c = 0; c < C; ++c) x[c] = (kbase + c > lim) ? -INFINITY : x[c] * sl2;
+          for (int c = 0; c < C; ++c)
+            x[c] = (kbase + c > lim || kbase + c < first) ? -INFINITY : x[c] * sl2;
         }
         // x holds raw scores (unmasked tile) or scaled, masked scores (masked tile).
         // exps(ms): p = 2^(x*sl2 - ms) (resp. 2^(x - ms)) for this group's C columns,
@@ -445,7 +502,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // the same named barriers; an abort is folded into the vote and forces the exact
         // path, which ends it. A NaN or infinite sum fails the compare and also goes
         // exact.
-        bool exact = (j == 0) || !(sl2 >= 0.f);
+        bool exact = (i == 0) || !(sl2 >= 0.f);
         if (!exact) {
           exps(m[t]);
           exact = named_bar_or(kBarVote, NTQ, !w_ok || !(rsum <= 256.f));
@@ -481,10 +538,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int g2 = 0; g2 < kFwdGroups; ++g2) mx = fmaxf(mx, xm[g2 * 128 + r]);
           const float m_new = fmaxf(m[t], mx);
           if (__any_sync(0xffffffffu, m_new > m[t] + 8.f)) {
-            const float alpha = ex2_approx(m[t] - m_new);  // 0 on the first tile (m = -inf)
+            // 0 while the row has seen no visible key (m = -inf; this also covers a row
+            // whose keys so far were all outside its window: -inf - -inf must not give NaN).
+            const float alpha = m[t] == -INFINITY ? 0.f : ex2_approx(m[t] - m_new);
             l[t] *= alpha;
             m[t] = m_new;
-            if (j > 0) {
+            if (i > 0) {
               // Rescale this group's D/G columns of the row's partial output before this
               // tile's products accumulate into it (PV_t(j-1) completed before S_t(j)).
 #pragma unroll
@@ -538,8 +597,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       constexpr int DG = D / kFwdGroups;  // output columns of this group
       const uint32_t tO = tmem + 256 + t * D + lane_off + grp * DG;
       const float inv_l = (lt > 0.f) ? 1.f / lt : 0.f;
-      const bool row_ok = row_g < p.N;
-      uint16_t* orow = p.out + ((static_cast<size_t>(b) * p.N + row_g) * p.H + h) * D + grp * DG;
+      const bool row_ok = row_g < seqlen;
+      const long long tok = (GENERAL && p.cu_seqlens != nullptr ? static_cast<long long>(seq0)
+                                                                : static_cast<long long>(b) * p.N) +
+                            row_g;
+      uint16_t* orow = p.out + tok * p.o_rs + h * D + grp * DG;
 #pragma unroll
       for (int cc = 0; cc < DG / 16; ++cc) {
         uint32_t o[16];
@@ -558,7 +620,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (row_ok && grp == 0) {
         const float lse = (lt > 0.f) ? (m[t] + log2f(lt)) * 0.69314718055994531f : -INFINITY;
-        p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + row_g] = lse;
+        if (GENERAL && p.cu_seqlens != nullptr)
+          p.lse[static_cast<size_t>(h) * p.total + tok] = lse;
+        else
+          p.lse[(static_cast<size_t>(b) * p.H + h) * p.N + row_g] = lse;
       }
     }
   }

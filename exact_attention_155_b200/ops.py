@@ -15,9 +15,9 @@ from typing import Optional, Tuple
 
 import torch
 
-__all__ = ["FAError", "load_library", "fwd", "bwd", "decode", "bwd_workspace_size",
-           "decode_workspace_size", "device_status", "debug_timeout_probe", "LIB_PATH",
-           "declared_symbols"]
+__all__ = ["FAError", "load_library", "fwd", "bwd", "fwd_ex", "bwd_ex", "fwd_qkvpacked",
+           "bwd_qkvpacked", "decode", "bwd_workspace_size", "decode_workspace_size",
+           "device_status", "debug_timeout_probe", "LIB_PATH", "declared_symbols"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
 
@@ -29,11 +29,20 @@ _c_void_p = ctypes.c_void_p
 _c_int = ctypes.c_int
 _c_float = ctypes.c_float
 _c_size_t = ctypes.c_size_t
+_c_ll = ctypes.c_longlong
 
 # name -> (restype, argtypes); mirrors include/fa.h
 _SIGNATURES = {
     "fa_fwd": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                         _c_int, _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p]),
+    "fa_fwd_ex": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                           _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
+                           _c_ll, _c_ll, _c_ll, _c_ll, _c_int, _c_int, _c_int, _c_float,
+                           _c_void_p]),
+    "fa_bwd_ex": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                           _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
+                           _c_int, _c_int, ctypes.POINTER(_c_ll), _c_int, _c_int, _c_int,
+                           _c_float, _c_void_p, _c_size_t, _c_void_p]),
     "fa_bwd_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
     "fa_bwd": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                         _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -191,6 +200,141 @@ def bwd(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = 
                                        workspace.numel(), _stream(stream),
                                        ctypes.c_void_p(ev0.cuda_event), ctypes.c_void_p(ev1.cuda_event)))
     return dq, dk, dv
+
+
+def _row_stride(t: torch.Tensor, name: str, varlen: bool, shape) -> int:
+    """Elements between consecutive tokens of a [B, N, H, d] (or [total, H, d]) view
+    whose (H, d) block is contiguous; raises for any other layout."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if t.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be torch.bfloat16 (got {t.dtype}); inputs and outputs share one dtype")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    H, d = shape[-2], shape[-1]
+    st = t.stride()
+    row = st[-3]
+    if st[-1] != 1 or (H > 1 and st[-2] != d):
+        raise ValueError(f"{name}: the (heads, head_dim) block of each row must be contiguous")
+    if not varlen and shape[0] > 1 and st[0] != shape[1] * row:
+        raise ValueError(f"{name}: batches must be N row strides apart")
+    return int(row)
+
+
+def _window(window):
+    wl, wr = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    return wl, wr
+
+
+def fwd_ex(q, k, v, causal: bool = False, scale: Optional[float] = None, window=None,
+           cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,
+           out=None, lse=None, stream=None):
+    """Forward with row strides, variable-length batches and a sliding window (fa_fwd_ex).
+
+    Dense: q, k, v are [B, N, H, d] views whose (H, d) block is contiguous (for example
+    slices of a packed [B, N, 3, H, d] tensor); lse is [B, H, N].
+    Variable length: q, k, v are [total, H, d]; cu_seqlens int32 [B + 1] on the device;
+    max_seqlen bounds every sequence length; lse is [H, total].
+    window = (left, right): query i sees keys [i - left, i + right], -1 = unbounded;
+    causal fixes right = 0. Returns (out, lse); out is contiguous unless given.
+    """
+    varlen = cu_seqlens is not None
+    if varlen:
+        _require(cu_seqlens, "cu_seqlens", torch.int32)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+            raise ValueError("cu_seqlens must be int32 [B + 1]")
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        total, H, d = q.shape
+        B, N = cu_seqlens.numel() - 1, int(max_seqlen)
+        shape = (total, H, d)
+    else:
+        B, N, H, d = q.shape
+        total = 0
+        shape = (B, N, H, d)
+    rs = [_row_stride(t, n, varlen, shape) for n, t in (("q", q), ("k", k), ("v", v))]
+    if out is None:
+        out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
+    rs.append(_row_stride(out, "out", varlen, shape))
+    lse_shape = (H, total) if varlen else (B, H, N)
+    if lse is None:
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
+    _require(lse, "lse", torch.float32)
+    if tuple(lse.shape) != lse_shape:
+        raise ValueError(f"lse must be {lse_shape}")
+    wl, wr = _window(window)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        _check(lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
+                             total, B, H, N, d, rs[0], rs[1], rs[2], rs[3], int(bool(causal)),
+                             wl, wr, _scale(scale, d), _stream(stream)))
+    return out, lse
+
+
+def bwd_ex(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = None,
+           window=None, cu_seqlens: Optional[torch.Tensor] = None,
+           max_seqlen: Optional[int] = None, dq=None, dk=None, dv=None, workspace=None,
+           stream=None):
+    """Backward of fwd_ex (fa_bwd_ex): same layouts and options. Returns (dq, dk, dv)."""
+    varlen = cu_seqlens is not None
+    if varlen:
+        _require(cu_seqlens, "cu_seqlens", torch.int32)
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        total, H, d = q.shape
+        B, N = cu_seqlens.numel() - 1, int(max_seqlen)
+        shape = (total, H, d)
+    else:
+        B, N, H, d = q.shape
+        total = 0
+        shape = (B, N, H, d)
+    dq = torch.empty(shape, dtype=torch.bfloat16, device=q.device) if dq is None else dq
+    dk = torch.empty(shape, dtype=torch.bfloat16, device=q.device) if dk is None else dk
+    dv = torch.empty(shape, dtype=torch.bfloat16, device=q.device) if dv is None else dv
+    names = (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq), ("dk", dk),
+             ("dv", dv))
+    rs = (_c_ll * 8)(*[_row_stride(t, n, varlen, shape) for n, t in names])
+    _require(lse, "lse", torch.float32)
+    lse_shape = (H, total) if varlen else (B, H, N)
+    if tuple(lse.shape) != lse_shape:
+        raise ValueError(f"lse must be {lse_shape}")
+    wl, wr = _window(window)
+    lib = load_library()
+    need = int(lib.fa_bwd_workspace_size(B, H, N, d))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        _check(lib.fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
+                             _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens), total, B, H, N, d, rs,
+                             int(bool(causal)), wl, wr, _scale(scale, d), _ptr(workspace),
+                             workspace.numel(), _stream(stream)))
+    return dq, dk, dv
+
+
+def fwd_qkvpacked(qkv, causal: bool = False, scale: Optional[float] = None, window=None,
+                  stream=None):
+    """Forward on a packed [B, N, 3, H, d] tensor (flash_attn_qkvpacked_func layout),
+    read in place through row strides. Returns (out [B, N, H, d], lse [B, H, N])."""
+    if qkv.dim() != 5 or qkv.shape[2] != 3:
+        raise ValueError("qkv must be [B, N, 3, H, d]")
+    _require(qkv, "qkv")
+    return fwd_ex(qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], causal=causal, scale=scale,
+                  window=window, stream=stream)
+
+
+def bwd_qkvpacked(qkv, out, dout, lse, causal: bool = False, scale: Optional[float] = None,
+                  window=None, dqkv=None, stream=None):
+    """Backward of fwd_qkvpacked; the gradient is written packed, [B, N, 3, H, d]."""
+    if qkv.dim() != 5 or qkv.shape[2] != 3:
+        raise ValueError("qkv must be [B, N, 3, H, d]")
+    _require(qkv, "qkv")
+    dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
+    _require(dqkv, "dqkv")
+    bwd_ex(qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], out, dout, lse, causal=causal, scale=scale,
+           window=window, dq=dqkv[:, :, 0], dk=dqkv[:, :, 1], dv=dqkv[:, :, 2], stream=stream)
+    return dqkv
 
 
 def decode_workspace_size(B: int, H: int, Ncap: int, d: int) -> int:

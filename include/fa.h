@@ -66,6 +66,38 @@ typedef enum {
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                  int B, int H, int N, int d, int causal, float scale, void* stream);
 
+/*
+ * Extended forward: the computation of fa_fwd with three generalisations.
+ *  - Row strides (packed QKV). Every row-major operand may have consecutive tokens
+ *    *_row_stride elements apart (a multiple of 8, at least H*d), so q, k and v can
+ *    be views into one packed [B, N, 3, H, d] tensor (q = base, k = base + H*d,
+ *    v = base + 2*H*d, row stride 3*H*d), the layout of flash_attn_qkvpacked_func in
+ *    "突破AI算力瓶颈：FlashAttention与MindSpore 2.0全场景融合方案" (核心API与使用示例).
+ *    Contiguous tensors have row stride H*d.
+ *  - Variable-length batches (packing, "ms-swift长文本训练优化，Flash-Attention显存省一半"
+ *    sections 4.2 and 5.1, flash_attn_varlen_func in section 4.3). With cu_seqlens
+ *    NULL the layout is the dense [B, N, H, d] (row (b, n) is token b*N + n) and lse
+ *    is [B, H, N]. With cu_seqlens (DEVICE int32 [B + 1], non-decreasing, cu[0] = 0,
+ *    cu[B] = total_tokens) the operands are [total_tokens, H, d], sequence b is
+ *    tokens [cu[b], cu[b+1]), N is an upper bound on every sequence length (it sizes
+ *    the grid), lse is [H, total_tokens], and attention never crosses sequences.
+ *    Entries that break these rules are reported as FA_ERR_DEVICE_INPUT through
+ *    fa_device_status and the affected sequences are left unwritten.
+ *    A tile that runs past the end of a sequence reads the next sequence's rows and
+ *    gives them probability 0: those rows must hold finite values (any finite values).
+ *  - Sliding window ("Flash-Attention 2/3在ms-swift中的集成与性能提升", FA3 feature
+ *    list: structured masks such as the sliding window). Query i sees keys
+ *    [i - window_left, i + window_right] within its sequence; -1 leaves that side
+ *    unbounded. causal != 0 is window_right = 0 (window_right must then be 0 or -1).
+ *    Key tiles outside every row's window are skipped, not masked.
+ * Errors as fa_fwd; a bad stride or window edge is FA_ERR_INVALID_ARG.
+ */
+fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* out, float* lse,
+                    const int* cu_seqlens, int total_tokens, int B, int H, int N, int d,
+                    long long q_row_stride, long long k_row_stride, long long v_row_stride,
+                    long long out_row_stride, int causal, int window_left, int window_right,
+                    float scale, void* stream);
+
 /* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator and
  * the per-row D = rowsum(dO * O) vector). Pure function of its arguments. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
@@ -100,6 +132,21 @@ fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const voi
                           int H, int N, int d, int causal, float scale, void* workspace,
                           size_t workspace_bytes, void* stream, void* main_start,
                           void* main_stop);
+
+/*
+ * Extended backward: the gradients of fa_fwd_ex, with the same row strides,
+ * variable-length batches and sliding window (see fa_fwd_ex). row_strides is a HOST
+ * array of 8 strides in elements, for q, k, v, out, dout, dq, dk, dv in that order
+ * (so dq, dk, dv can be views into one packed [B, N, 3, H, d] gradient). lse is the
+ * forward's ([B, H, N] dense, [H, total_tokens] variable length). The workspace is
+ * fa_bwd_workspace_size(B, H, N, d) bytes with N the largest sequence length.
+ * Errors as fa_bwd and fa_fwd_ex.
+ */
+fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens,
+                    int total_tokens, int B, int H, int N, int d, const long long* row_strides,
+                    int causal, int window_left, int window_right, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream);
 
 /*
  * fa_bwd for callers that cannot allocate device memory. Some callers have no way
