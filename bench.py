@@ -26,6 +26,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import itertools
 import json
 import math
 import os
@@ -233,7 +234,8 @@ def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
     import exact_attention_155_b200 as fa
-    from exact_attention_155_b200.inputs import attention_inputs, decode_inputs
+    from exact_attention_155_b200.inputs import (VARLEN_BENCH, WINDOW_BENCH, attention_inputs,
+                                                 bf16_randn, decode_inputs, packed_lengths)
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -448,6 +450,50 @@ def run_ours(args, rank, world, local_rank):
         graph.replay()
         gms = timed_events(torch, graph.replay, 10)
         del graph
+        del kc, vc, qs, ks, vs, o5, l5, ws5
+        # Sliding-window causal attention (window 4096) on a 16K sequence, fwd and bwd.
+        wb = WINDOW_BENCH
+        win = attention_inputs(wb["B"], wb["N"], wb["H"], wb["d"], seed=wb["seed"])
+        wq, wk, wv, wdo = (win[n].to(dev) for n in ("q", "k", "v", "dout"))
+        del win
+        wwin = wb["window"]
+        wo, wlse = fa.fwd_ex(wq, wk, wv, causal=True, scale=scale, window=wwin)
+        wg = [torch.empty_like(wq) for _ in range(3)]
+        wws = torch.empty(fa.bwd_workspace_size(wb["B"], wb["H"], wb["N"], wb["d"]),
+                          dtype=torch.uint8, device=dev)
+        fwd_w = lambda: fa.fwd_ex(wq, wk, wv, causal=True, scale=scale, window=wwin, out=wo, lse=wlse)
+        bwd_w = lambda: fa.bwd_ex(wq, wk, wv, wo, wdo, wlse, causal=True, scale=scale, window=wwin,
+                                  dq=wg[0], dk=wg[1], dv=wg[2], workspace=wws)
+        for _ in range(3):
+            fwd_w()
+            bwd_w()
+        wf_ms = timed_events(torch, fwd_w, 10)
+        wb_ms = timed_events(torch, bwd_w, 10)
+        w_left = wwin[0]
+        pairs = w_left * (w_left + 1) // 2 + (wb["N"] - w_left) * (w_left + 1)  # visible (q, k)
+        wf_fl = 4.0 * wb["d"] * wb["B"] * wb["H"] * pairs
+        del wq, wk, wv, wdo, wo, wlse, wg, wws
+        # Packed variable-length batch (seeded length mix), causal, fwd and bwd.
+        vb = VARLEN_BENCH
+        lens = packed_lengths(vb["total"], vb["lo"], vb["hi"], vb["seed"])
+        cu = torch.tensor([0] + list(itertools.accumulate(lens)), dtype=torch.int32, device=dev)
+        gen = torch.Generator().manual_seed(vb["seed"])
+        vq, vk, vv, vdo = (bf16_randn((vb["total"], vb["H"], vb["d"]), gen).to(dev) for _ in range(4))
+        vo, vlse = fa.fwd_ex(vq, vk, vv, causal=True, scale=scale, cu_seqlens=cu, max_seqlen=max(lens))
+        vg = [torch.empty_like(vq) for _ in range(3)]
+        vws = torch.empty(fa.bwd_workspace_size(len(lens), vb["H"], max(lens), vb["d"]),
+                          dtype=torch.uint8, device=dev)
+        fwd_v = lambda: fa.fwd_ex(vq, vk, vv, causal=True, scale=scale, cu_seqlens=cu,
+                                  max_seqlen=max(lens), out=vo, lse=vlse)
+        bwd_v = lambda: fa.bwd_ex(vq, vk, vv, vo, vdo, vlse, causal=True, scale=scale, cu_seqlens=cu,
+                                  max_seqlen=max(lens), dq=vg[0], dk=vg[1], dv=vg[2], workspace=vws)
+        for _ in range(3):
+            fwd_v()
+            bwd_v()
+        vf_ms = timed_events(torch, fwd_v, 10)
+        vb_ms = timed_events(torch, bwd_v, 10)
+        vf_fl = 4.0 * vb["d"] * vb["H"] * sum(n * (n + 1) // 2 for n in lens)
+        del vq, vk, vv, vdo, vo, vlse, vg, vws
         parts = {
             "prefill_fwd": {"workload": "causal fwd B=1 H=32 N=8192 d=128", "value": ptf,
                             "unit": "TFLOP/s", "ms": pms, "roofline_bound": "tensor",
@@ -461,6 +507,24 @@ def run_ours(args, rank, world, local_rank):
                              "roofline_bound": "hbm", "frac": dgbs / peaks["hbm"],
                              "peak": peaks["hbm"], "peak_kind": f"HBM copy, of {peaks['source']}",
                              "l2": "flushed before every call (512 MiB write, then 256 MiB read)"},
+            "window_causal": {
+                "workload": f"causal sliding window {wwin[0]}, B=1 H=32 N=16384 d=128",
+                "fwd_tflops": wf_fl / (wf_ms * 1e-3) / 1e12, "fwd_ms": wf_ms,
+                "bwd_tflops": 2.5 * wf_fl / (wb_ms * 1e-3) / 1e12, "bwd_ms": wb_ms,
+                "flop_count": "4*d*H per visible (query, key) pair, x2.5 for bwd",
+                "bwd_includes": "preprocess, main and dq-convert kernels",
+                "roofline_bound": "tensor",
+                "fwd_frac": wf_fl / (wf_ms * 1e-3) / 1e12 / peaks["tf_burst"],
+                "peak": peaks["tf_burst"], "peak_kind": f"bf16 dense, burst, of {peaks['source']}"},
+            "varlen_causal": {
+                "workload": f"packed causal batch, {len(lens)} sequences of {min(lens)}-{max(lens)} tokens "
+                            f"({vb['total']} tokens), H=32 d=128",
+                "fwd_tflops": vf_fl / (vf_ms * 1e-3) / 1e12, "fwd_ms": vf_ms,
+                "bwd_tflops": 2.5 * vf_fl / (vb_ms * 1e-3) / 1e12, "bwd_ms": vb_ms,
+                "bwd_includes": "preprocess, main and dq-convert kernels",
+                "roofline_bound": "tensor",
+                "fwd_frac": vf_fl / (vf_ms * 1e-3) / 1e12 / peaks["tf_burst"],
+                "peak": peaks["tf_burst"], "peak_kind": f"bf16 dense, burst, of {peaks['source']}"},
             "decode_steps": {"workload": "decode B=2 H=16 d=64 cap 2048, 100 appending steps",
                              "us_per_step": sms * 1e3 / c5["steps"],
                              "us_per_step_cuda_graph": gms * 1e3 / c5["steps"],

@@ -53,6 +53,27 @@ DECODE_STEPS = dict(B=2, H=16, d=64, Ncap=2048, steps=100, config_id=5)
 DECODE_SWEEP = dict(B=32, H=16, d=64, Ncap=2048, seqlen=2048, config_id=5)
 
 
+# Sliding-window workload: long causal sequence, local window of 4096 keys.
+WINDOW_BENCH = dict(B=1, H=32, N=16384, d=128, window=(4096, 0), seed=1007)
+# Packed variable-length workload: the packing example of the long-text page (samples
+# of 1-2K tokens packed instead of padded) stood in for by seeded lengths drawn
+# uniformly from [512, 4096] until 32768 tokens are filled (the last one is cut).
+VARLEN_BENCH = dict(total=32768, H=32, d=128, lo=512, hi=4096, seed=1006)
+
+
+def packed_lengths(total: int, lo: int, hi: int, seed: int):
+    """Seeded sequence lengths in [lo, hi] summing to exactly `total`."""
+    g = torch.Generator().manual_seed(int(seed))
+    lens = []
+    left = total
+    while left > 0:
+        n = int(torch.randint(lo, hi + 1, (1,), generator=g))
+        n = min(n, left)
+        lens.append(n)
+        left -= n
+    return lens
+
+
 def seed_for(config_id: int) -> int:
     return 1000 + int(config_id)
 

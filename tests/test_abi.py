@@ -89,6 +89,43 @@ def test_bwd_argument_errors(lib):
     assert _bwd(lib, scale=math.inf) == INVALID
 
 
+def _fwd_ex(lib, cu=NULL, total=0, B=1, H=2, N=128, d=64, rs=(128, 128, 128, 128), causal=0,
+            wl=-1, wr=-1, scale=0.125, q=P16):
+    return lib.fa_fwd_ex(q, P16, P16, P16, P16, cu, total, B, H, N, d, *rs, causal, wl, wr, scale,
+                         NULL)
+
+
+def test_fwd_ex_argument_errors(lib):
+    # Row strides: a multiple of 8 elements and at least H*d.
+    assert _fwd_ex(lib, rs=(128, 128, 120, 128)) == INVALID
+    assert b"stride" in lib.fa_last_error()
+    assert _fwd_ex(lib, rs=(132, 128, 128, 128)) == INVALID
+    # Window edges: >= 0 or -1; causal allows only a right edge of 0 or -1.
+    assert _fwd_ex(lib, wl=-2) == INVALID
+    assert _fwd_ex(lib, causal=1, wr=5) == INVALID
+    assert b"window_right" in lib.fa_last_error()
+    assert _fwd_ex(lib, d=80) == UNSUPPORTED
+    assert _fwd_ex(lib, q=NULL) == INVALID
+    assert _fwd_ex(lib, scale=math.nan) == INVALID
+    # A packed batch with no tokens, or no sequences, is a no-op.
+    assert _fwd_ex(lib, cu=P16, total=0) == FA_OK
+    assert _fwd_ex(lib, B=0) == FA_OK
+
+
+def test_bwd_ex_argument_errors(lib):
+    rs8 = (ctypes.c_longlong * 8)(*([128] * 8))
+
+    def call(rs=rs8, ws=P16, ws_bytes=1 << 30, wr=-1, causal=0):
+        return lib.fa_bwd_ex(P16, P16, P16, P16, P16, P16, P16, P16, P16, NULL, 0, 1, 2, 128, 64,
+                             rs, causal, -1, wr, 0.125, ws, ws_bytes, NULL)
+
+    assert call(rs=None) == INVALID
+    bad = (ctypes.c_longlong * 8)(*([128] * 7 + [100]))
+    assert call(rs=bad) == INVALID
+    assert call(causal=1, wr=3) == INVALID
+    assert call(ws=NULL) == WORKSPACE
+
+
 def _dec(lib, q=P16, kn=NULL, vn=NULL, seq=P16, Ncap=2048, d=64, B=2):
     return lib.fa_decode(q, P16, P16, seq, kn, vn, P16, NULL, B, 16, Ncap, d, 1, 0.125, NULL, 0, S0)
 

@@ -153,3 +153,56 @@ def test_bad_cu_seqlens_are_reported_on_the_device():
                                                    scale=default_scale(d))
         got = out[:10].float().cpu().numpy()
         assert np.max(np.abs(got - ref_o)) <= OUT_ATOL
+
+
+def test_window_bench_size_sampled():
+    """The sliding-window workload bench.py times (B=1 H=32 N=16384 d=128, causal,
+    window 4096), in the same launch; the oracle recomputes heads 0 and 31 (forward on
+    sampled rows, backward on all rows of head 0)."""
+    from exact_attention_155_b200.inputs import WINDOW_BENCH as wb
+    inp = make_inputs(wb["B"], wb["N"], wb["H"], wb["d"], wb["seed"])
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    sc = default_scale(wb["d"])
+    wl, wr = wb["window"]
+    out, lse = fa.fwd_ex(q, k, v, causal=True, scale=sc, window=(wl, wr))
+    grads = fa.bwd_ex(q, k, v, out, do, lse, causal=True, scale=sc, window=(wl, wr))
+    torch.cuda.synchronize()
+    rows = sorted(set(list(range(0, wb["N"], 97)) + list(range(wb["N"] - 130, wb["N"]))
+                      + list(range(wl - 3, wl + 130))))
+    qf, kf, vf, dof = (to_f64(inp[n]) for n in ("q", "k", "v", "dout"))
+    ref_o, ref_l = oracle.attention_forward(qf, kf, vf, causal=True, scale=sc, heads=[(0, 0), (0, 31)],
+                                            rows=rows, window_left=wl, window_right=wr)
+    m = ~np.isnan(ref_o)
+    got = out.float().cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got[m] - ref_o[m])) <= OUT_ATOL
+    ml = ~np.isnan(ref_l)
+    assert np.max(np.abs(lse.cpu().numpy()[ml] - ref_l[ml])) <= LSE_ATOL
+    refs = oracle.attention_backward(qf, kf, vf, dof, causal=True, scale=sc, heads=[(0, 0)],
+                                     window_left=wl, window_right=wr)
+    for name, g, r in zip(("dq", "dk", "dv"), grads, refs):
+        mm = ~np.isnan(r)
+        gg = g.float().cpu().numpy().astype(np.float64)
+        assert np.max(np.abs(gg[mm] - r[mm])) <= GRAD_REL * np.max(np.abs(r[mm])), name
+
+
+def test_varlen_bench_size_sampled():
+    """The packed variable-length workload bench.py times (32768 tokens, H=32, d=128,
+    causal), in the same launch; the oracle recomputes heads 0 and 31 of every sequence."""
+    from exact_attention_155_b200.inputs import VARLEN_BENCH as vb, packed_lengths
+    lens = packed_lengths(vb["total"], vb["lo"], vb["hi"], vb["seed"])
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    g = torch.Generator().manual_seed(vb["seed"])
+    q, k, v, do = (bf16_randn((vb["total"], vb["H"], vb["d"]), g) for _ in range(4))
+    sc = default_scale(vb["d"])
+    cu_t = torch.from_numpy(cu).cuda()
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, do))
+    out, lse = fa.fwd_ex(qc, kc, vc, causal=True, scale=sc, cu_seqlens=cu_t, max_seqlen=max(lens))
+    grads = fa.bwd_ex(qc, kc, vc, out, doc, lse, causal=True, scale=sc, cu_seqlens=cu_t,
+                      max_seqlen=max(lens))
+    torch.cuda.synchronize()
+    hs = [0, vb["H"] - 1]
+    sub = lambda t: to_f64(t[:, hs])
+    ref_o, ref_l = oracle.attention_forward_varlen(sub(q), sub(k), sub(v), cu, causal=True, scale=sc)
+    _cmp_out(out[:, hs], lse[hs], ref_o, ref_l)
+    refs = oracle.attention_backward_varlen(sub(q), sub(k), sub(v), sub(do), cu, causal=True, scale=sc)
+    _cmp_grads(tuple(gr[:, hs] for gr in grads), refs)
