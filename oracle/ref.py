@@ -40,6 +40,11 @@ Readings taken where the pages are silent (each is also listed in the design not
   the page names the mask, not its parameters): with the query's position on the key
   axis i' = i + (Nk - Nq), key j is visible iff i' - window_left <= j <= i' +
   window_right; -1 leaves a side unbounded. It combines with the causal mask by AND.
+* Paged KV cache ("突破AI算力瓶颈：FlashAttention与MindSpore 2.0全场景融合方案",
+  section 推理优化与KV缓存: the cache is stored in pages to avoid fragmentation): pages
+  of page_size rows are [num_pages, page_size, H, d]; row r of sequence b is row
+  r % page_size of page block_table[b][r // page_size]. Paging is addressing only:
+  the step is the contiguous decode step on the rows the table names.
 * Variable-length batches (packing, "ms-swift长文本训练优化，Flash-Attention显存省一半"
   sections 4.2 and 5.1): tokens of B sequences are packed into [total, H, d] and
   sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]); each sequence is an
@@ -71,6 +76,7 @@ __all__ = [
     "merge_partials",
     "decode_step",
     "decode_sequence",
+    "decode_step_paged",
 ]
 
 
@@ -375,6 +381,32 @@ def decode_step(q, k_cache, v_cache, cache_seqlens, k_new=None, v_new=None,
             out[b, 0, h] = (p @ vc[b, :L, h, :])[0]
             lse[b, h] = l[0]
     return out, lse, kc, vc
+
+
+def decode_step_paged(q, k_pages, v_pages, block_table, cache_seqlens, k_new=None, v_new=None,
+                      scale=None):
+    """decode_step over a paged cache: gather each sequence's logical rows through its
+    block table, run decode_step, and scatter the appended row back into its page.
+
+    k_pages, v_pages: [num_pages, page_size, H, d]; block_table: int [B, max_blocks].
+    Returns (out [B, 1, H, d], lse [B, H], k_pages', v_pages') with the pages copied.
+    """
+    kp = np.array(k_pages, dtype=np.float64, copy=True)
+    vp = np.array(v_pages, dtype=np.float64, copy=True)
+    bt = np.asarray(block_table)
+    B, max_blocks = bt.shape
+    P = kp.shape[1]
+    rows = np.arange(max_blocks * P)
+    page_of, slot_of = rows // P, rows % P
+    kc = np.stack([kp[bt[b, page_of], slot_of] for b in range(B)])  # [B, cap, H, d]
+    vc = np.stack([vp[bt[b, page_of], slot_of] for b in range(B)])
+    out, lse, kc2, vc2 = decode_step(q, kc, vc, cache_seqlens, k_new, v_new, scale=scale)
+    if k_new is not None:
+        for b in range(B):
+            r = int(cache_seqlens[b])
+            kp[bt[b, r // P], r % P] = kc2[b, r]
+            vp[bt[b, r // P], r % P] = vc2[b, r]
+    return out, lse, kp, vp
 
 
 def decode_sequence(q_steps, k_steps, v_steps, k_cache, v_cache, start_seqlens,

@@ -160,3 +160,44 @@ def test_window_pin_catches_planted_off_by_one(monkeypatch):
     out, _ = ref.attention_forward(q, k, v, scale=0.7, window_left=2, window_right=0)
     bo, _ = _brute(q, k, v, False, 0.7, 2, 0)
     assert not np.allclose(out[0], bo, atol=1e-6)
+
+
+# ------------------------------------------------------------------- paged KV cache
+
+
+def _paged_from_contiguous(kc, P, perm):
+    """Split a contiguous [B, cap, H, d] cache into pages placed at `perm` positions."""
+    B, cap, H, d = kc.shape
+    nb = cap // P
+    pages = np.full((B * nb + 3, P, H, d), np.nan)  # spare pages stay NaN: never read
+    table = np.zeros((B, nb), dtype=np.int64)
+    for b in range(B):
+        for j in range(nb):
+            pid = perm[b * nb + j]
+            pages[pid] = kc[b, j * P:(j + 1) * P]
+            table[b, j] = pid
+    return pages, table
+
+
+def test_paged_decode_is_contiguous_decode_under_any_page_placement():
+    B, cap, H, d, P = 3, 64, 2, 8, 16
+    kc, vc = _rand((B, cap, H, d), 90), _rand((B, cap, H, d), 91)
+    q, kn, vn = _rand((B, 1, H, d), 92), _rand((B, 1, H, d), 93), _rand((B, 1, H, d), 94)
+    seq = np.array([0, 37, 63])
+    ref_o, ref_l, ref_k, _ = oracle.decode_step(q, kc, vc, seq, kn, vn, scale=0.3)
+    perm = np.random.default_rng(95).permutation(B * (cap // P) + 3)
+    kp, table = _paged_from_contiguous(kc, P, perm)
+    vp, _ = _paged_from_contiguous(vc, P, perm)
+    o, l, kp2, _ = oracle.decode_step_paged(q, kp, vp, table, seq, kn, vn, scale=0.3)
+    np.testing.assert_array_equal(o, ref_o)
+    np.testing.assert_array_equal(l, ref_l)
+    # The appended row landed in its page, at the slot its position names.
+    for b in range(B):
+        r = seq[b]
+        np.testing.assert_array_equal(kp2[table[b, r // P], r % P], kn[b, 0])
+    # Spare pages were neither read (outputs finite) nor written.
+    spare = sorted(set(range(kp.shape[0])) - set(table.ravel().tolist()))
+    assert np.isnan(kp2[spare]).all()
+    assert np.isfinite(o).all()
+    # Step 0 of sequence 0 returns the new value row exactly.
+    np.testing.assert_array_equal(o[0, 0], vn[0, 0])
