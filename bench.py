@@ -422,7 +422,22 @@ def run_ours(args, rank, world, local_rank):
         dms = timed_events(torch, dec, 30, flush=flush)
         dbytes = 2 * s["B"] * s["H"] * s["seqlen"] * s["d"] * 2
         dgbs = dbytes / (dms * 1e-3) / 1e9
-        del kc, vc, flush_w, flush_r
+        # The same sweep over a paged cache: 64-row pages at shuffled pool positions.
+        page = 64
+        nb = s["Ncap"] // page
+        gperm = torch.Generator().manual_seed(1008)
+        perm = torch.randperm(s["B"] * nb, generator=gperm).to(dev)
+        table = perm.view(s["B"], nb).to(torch.int32)
+        kp = torch.empty((s["B"] * nb, page, s["H"], s["d"]), dtype=torch.bfloat16, device=dev)
+        vp = torch.empty_like(kp)
+        kp[perm] = kc.view(s["B"] * nb, page, s["H"], s["d"])
+        vp[perm] = vc.view(s["B"] * nb, page, s["H"], s["d"])
+        decp = lambda: fa.decode_paged(qd, kp, vp, table, seq, scale=1 / 8, out=dout_, lse=dlse)
+        for _ in range(3):
+            decp()
+        pdms = timed_events(torch, decp, 30, flush=flush)
+        pdgbs = dbytes / (pdms * 1e-3) / 1e9
+        del kc, vc, kp, vp, table, flush_w, flush_r
         c5 = STEPS5
         kc, vc, qs, ks, vs = decode_inputs(c5["B"], c5["H"], c5["d"], c5["Ncap"], c5["steps"], seed=1005)
         kc, vc, qs, ks, vs = kc.to(dev), vc.to(dev), qs.to(dev), ks.to(dev), vs.to(dev)
@@ -507,6 +522,13 @@ def run_ours(args, rank, world, local_rank):
                              "roofline_bound": "hbm", "frac": dgbs / peaks["hbm"],
                              "peak": peaks["hbm"], "peak_kind": f"HBM copy, of {peaks['source']}",
                              "l2": "flushed before every call (512 MiB write, then 256 MiB read)"},
+            "decode_sweep_paged": {"workload": "decode B=32 H=16 d=64, 2048 rows in 64-row pages "
+                                               "at shuffled pool positions, no append",
+                                   "value": pdgbs, "unit": "GB/s", "us": pdms * 1e3,
+                                   "roofline_bound": "hbm", "frac": pdgbs / peaks["hbm"],
+                                   "peak": peaks["hbm"],
+                                   "peak_kind": f"HBM copy, of {peaks['source']}",
+                                   "l2": "flushed before every call"},
             "window_causal": {
                 "workload": f"causal sliding window {wwin[0]}, B=1 H=32 N=16384 d=128",
                 "fwd_tflops": wf_fl / (wf_ms * 1e-3) / 1e12, "fwd_ms": wf_ms,

@@ -6,7 +6,9 @@ example for its seeded input generators) needs no GPU. Calls raise if the librar
 is missing or the device is not sm_100.
 """
 from .ops import (FAError, bwd, bwd_ex, bwd_qkvpacked, bwd_workspace_size, decode,  # noqa: F401
-                  decode_workspace_size, device_status, fwd, fwd_ex, fwd_qkvpacked, load_library)
+                  decode_paged, decode_workspace_size, device_status, fwd, fwd_ex, fwd_qkvpacked,
+                  load_library)
 
 __all__ = ["FAError", "fwd", "bwd", "fwd_ex", "bwd_ex", "fwd_qkvpacked", "bwd_qkvpacked", "decode",
+           "decode_paged",
            "bwd_workspace_size", "decode_workspace_size", "device_status", "load_library"]

@@ -49,9 +49,14 @@ struct DecodeParams {
   float* lse;             // [B, H] or null
   int B, H, Ncap, nsplit, chunk;
   float scale_log2;
+  // Paged caches (decode_kernel<D, true>): k_cache / v_cache are [num_pages, page_size,
+  // H, d]; row r of batch b is row r % page_size of page block_table[b][r / page_size].
+  // Ncap = max_blocks * page_size is the logical capacity.
+  const int* block_table;  // [B, max_blocks]
+  int max_blocks, num_pages, page_shift;  // page_size = 1 << page_shift
 };
 
-enum : unsigned int { kSiteDecodeSeqlen = 0x301 };
+enum : unsigned int { kSiteDecodeSeqlen = 0x301, kSiteDecodePage = 0x302 };
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
   const uint32_t w[4] = {u.x, u.y, u.z, u.w};
@@ -81,7 +86,7 @@ __device__ __forceinline__ void online_merge(float& m, float& l, float (&o)[8], 
 // thread-block cluster and combine their partial states in the leader CTA's shared
 // memory (distributed shared memory), so the whole step is a single launch with no
 // global workspace.
-template <int D>
+template <int D, bool PAGED>
 __global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
   constexpr int LPR = D / 8;     // lanes per cache row (16 bytes each)
   constexpr int RPW = 32 / LPR;  // rows per warp per step
@@ -111,19 +116,37 @@ __global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
   const int k1 = min(k0 + p.chunk, Lt);
   const size_t bh = static_cast<size_t>(b) * p.H + h;
   const size_t row_stride = static_cast<size_t>(p.H) * D;  // elements between cache rows
-  const uint16_t* kc = p.k_cache + (static_cast<size_t>(b) * p.Ncap * p.H + h) * D + sub * 8;
-  const uint16_t* vc = p.v_cache + (static_cast<size_t>(b) * p.Ncap * p.H + h) * D + sub * 8;
+  const size_t cache0 = PAGED ? static_cast<size_t>(h) * D
+                              : (static_cast<size_t>(b) * p.Ncap * p.H + h) * D;
+  const uint16_t* kc = p.k_cache + cache0 + sub * 8;
+  const uint16_t* vc = p.v_cache + cache0 + sub * 8;
+  // Element offset of cache row r from this (b, h)'s row 0 (contiguous) or from the
+  // cache base (paged), or -1 for a page id outside [0, num_pages), which is reported
+  // and never dereferenced.
+  auto row_off = [&](int r) -> long long {
+    if (!PAGED) return static_cast<long long>(r) * static_cast<long long>(row_stride);
+    const int pg = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + (r >> p.page_shift));
+    if (pg < 0 || pg >= p.num_pages) {
+      report(kDevBadInput, kSiteDecodePage, b);
+      return -1;
+    }
+    return ((static_cast<long long>(pg) << p.page_shift) + (r & ((1 << p.page_shift) - 1))) *
+           static_cast<long long>(row_stride);
+  };
   const uint16_t* kn = append ? p.k_new + bh * D + sub * 8 : nullptr;
   const uint16_t* vn = append ? p.v_new + bh * D + sub * 8 : nullptr;
 
   // The CTA whose chunk holds the appended row persists it in the cache; every CTA
   // reads that row from k_new / v_new, never from the cache.
   if (do_append && L >= k0 && L < k1 && tid < LPR) {
-    const size_t off = (static_cast<size_t>(b) * p.Ncap + L) * row_stride + h * D + tid * 8;
-    *reinterpret_cast<uint4*>(p.k_cache + off) =
-        *reinterpret_cast<const uint4*>(p.k_new + bh * D + tid * 8);
-    *reinterpret_cast<uint4*>(p.v_cache + off) =
-        *reinterpret_cast<const uint4*>(p.v_new + bh * D + tid * 8);
+    const long long ro = row_off(L);
+    if (ro >= 0) {
+      const size_t off = cache0 + static_cast<size_t>(ro) + tid * 8;
+      *reinterpret_cast<uint4*>(p.k_cache + off) =
+          *reinterpret_cast<const uint4*>(p.k_new + bh * D + tid * 8);
+      *reinterpret_cast<uint4*>(p.v_cache + off) =
+          *reinterpret_cast<const uint4*>(p.v_new + bh * D + tid * 8);
+    }
   }
 
   float qf[8];
@@ -141,16 +164,21 @@ __global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
   // Rows handled by this lane group: k0 + warp*RPW + grp + RSTEP*t, t = 0, 1, ...
   for (int base = k0 + warp * RPW; base < k1; base += U * RSTEP) {
     uint4 kv[U], vv[U];
+    bool live[U];  // row inside the chunk with a readable source
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int kb = base + u * RSTEP + grp;
       kv[u] = make_uint4(0, 0, 0, 0);
       vv[u] = make_uint4(0, 0, 0, 0);
+      live[u] = false;
       if (kb < k1) {
         const bool is_new = do_append && kb == L;
-        const size_t off = static_cast<size_t>(kb) * row_stride;
-        kv[u] = __ldg(reinterpret_cast<const uint4*>(is_new ? kn : kc + off));
-        vv[u] = __ldg(reinterpret_cast<const uint4*>(is_new ? vn : vc + off));
+        const long long off = is_new ? 0 : row_off(kb);
+        if (is_new || off >= 0) {
+          live[u] = true;
+          kv[u] = __ldg(reinterpret_cast<const uint4*>(is_new ? kn : kc + off));
+          vv[u] = __ldg(reinterpret_cast<const uint4*>(is_new ? vn : vc + off));
+        }
       }
     }
     float sc[U];
@@ -163,7 +191,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
       for (int i = 0; i < 8; ++i) acc = fmaf(qf[i], f[i], acc);
 #pragma unroll
       for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-      sc[u] = (base + u * RSTEP + grp < k1) ? acc : -INFINITY;
+      sc[u] = live[u] ? acc : -INFINITY;
     }
     float mx = sc[0];
 #pragma unroll

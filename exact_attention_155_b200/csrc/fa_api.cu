@@ -569,32 +569,36 @@ size_t fa_decode_workspace_size(int B, int H, int Ncap, int d) {
   return 0;  // split partials are combined on chip (cluster shared memory)
 }
 
-fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cache_seqlens,
-                    const void* k_new, const void* v_new, void* out, float* lse, int B, int H,
-                    int Ncap, int d, int causal, float scale, void* workspace,
-                    size_t workspace_bytes, void* stream) {
-  (void)causal;  // one query at the end of the sequence sees every valid key
-  if (B < 0 || H < 0) return fail(FA_ERR_INVALID_ARG, "fa_decode: negative size B=%d H=%d", B, H);
-  if (Ncap <= 0) return fail(FA_ERR_INVALID_ARG, "fa_decode: cache capacity must be >= 1 (got %d)", Ncap);
-  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "fa_decode: head dim %d not supported (64 or 128)", d);
-  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "fa_decode: scale must be finite");
+}  // extern "C"
+
+namespace {
+
+// Shared by fa_decode and fa_decode_paged: argument checks, split choice and the
+// cluster launch. block_table == NULL selects the contiguous cache layout.
+fa_status run_decode(const char* who, const void* q, void* k_cache, void* v_cache,
+                     const int* cache_seqlens, const void* k_new, const void* v_new, void* out,
+                     float* lse, int B, int H, int Ncap, int d, float scale,
+                     const int* block_table, int max_blocks, int page_shift, int num_pages,
+                     void* stream) {
+  if (B < 0 || H < 0) return fail(FA_ERR_INVALID_ARG, "%s: negative size B=%d H=%d", who, B, H);
+  if (Ncap <= 0) return fail(FA_ERR_INVALID_ARG, "%s: cache capacity must be >= 1 (got %d)", who, Ncap);
+  if (d != 64 && d != 128) return fail(FA_ERR_UNSUPPORTED, "%s: head dim %d not supported (64 or 128)", who, d);
+  if (!std::isfinite(scale)) return fail(FA_ERR_INVALID_ARG, "%s: scale must be finite", who);
   if (B == 0 || H == 0) return FA_OK;
   if (!q || !k_cache || !v_cache || !cache_seqlens || !out)
-    return fail(FA_ERR_INVALID_ARG, "fa_decode: null pointer");
+    return fail(FA_ERR_INVALID_ARG, "%s: null pointer", who);
   if ((k_new == nullptr) != (v_new == nullptr))
-    return fail(FA_ERR_INVALID_ARG, "fa_decode: k_new and v_new must both be given or both be NULL");
+    return fail(FA_ERR_INVALID_ARG, "%s: k_new and v_new must both be given or both be NULL", who);
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
       (k_new && (!aligned16(k_new) || !aligned16(v_new))) || !aligned4(cache_seqlens) ||
-      (lse && !aligned4(lse)))
-    return fail(FA_ERR_INVALID_ARG, "fa_decode: bf16 tensors must be 16-byte aligned, int/float 4-byte");
-  if (H > 65535 || B > 65535) return fail(FA_ERR_INVALID_ARG, "fa_decode: B and H must be <= 65535");
+      (lse && !aligned4(lse)) || (block_table && !aligned4(block_table)))
+    return fail(FA_ERR_INVALID_ARG, "%s: bf16 tensors must be 16-byte aligned, int/float 4-byte", who);
+  if (H > 65535 || B > 65535) return fail(FA_ERR_INVALID_ARG, "%s: B and H must be <= 65535", who);
   int dev = 0, sms = 0;
   fa_status st = current_device(&dev, &sms);
   if (st != FA_OK) return st;
   int chunk = 0;
   const int ns = decode_splits(B, H, Ncap, sms, &chunk);
-  (void)workspace;
-  (void)workspace_bytes;
   fa::DecodeParams p;
   p.q = static_cast<const uint16_t*>(q);
   p.k_cache = static_cast<uint16_t*>(k_cache);
@@ -610,6 +614,10 @@ fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cach
   p.nsplit = ns;
   p.chunk = chunk;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.block_table = block_table;
+  p.max_blocks = max_blocks;
+  p.num_pages = num_pages;
+  p.page_shift = page_shift;
   // The `ns` CTAs of one (batch, head) run as one thread-block cluster.
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ns, H, B);
@@ -623,10 +631,50 @@ fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cach
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = (d == 64) ? cudaLaunchKernelEx(&cfg, fa::decode_kernel<64>, p)
-                            : cudaLaunchKernelEx(&cfg, fa::decode_kernel<128>, p);
-  if (e != cudaSuccess) return cuda_fail(e, "fa_decode kernel launch");
-  return check_launch("fa_decode kernel launch");
+  cudaError_t e;
+  if (block_table)
+    e = (d == 64) ? cudaLaunchKernelEx(&cfg, fa::decode_kernel<64, true>, p)
+                  : cudaLaunchKernelEx(&cfg, fa::decode_kernel<128, true>, p);
+  else
+    e = (d == 64) ? cudaLaunchKernelEx(&cfg, fa::decode_kernel<64, false>, p)
+                  : cudaLaunchKernelEx(&cfg, fa::decode_kernel<128, false>, p);
+  if (e != cudaSuccess) return cuda_fail(e, "decode kernel launch");
+  return check_launch("decode kernel launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cache_seqlens,
+                    const void* k_new, const void* v_new, void* out, float* lse, int B, int H,
+                    int Ncap, int d, int causal, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream) {
+  (void)causal;  // one query at the end of the sequence sees every valid key
+  (void)workspace;
+  (void)workspace_bytes;
+  return run_decode("fa_decode", q, k_cache, v_cache, cache_seqlens, k_new, v_new, out, lse, B, H,
+                    Ncap, d, scale, nullptr, 0, 0, 0, stream);
+}
+
+fa_status fa_decode_paged(const void* q, void* k_pages, void* v_pages, const int* block_table,
+                          int max_blocks, int page_size, int num_pages, const int* cache_seqlens,
+                          const void* k_new, const void* v_new, void* out, float* lse, int B,
+                          int H, int d, int causal, float scale, void* stream) {
+  (void)causal;
+  if (page_size < 1 || page_size > (1 << 16) || (page_size & (page_size - 1)) != 0)
+    return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: page_size must be a power of two in [1, 65536] (got %d)",
+                page_size);
+  if (max_blocks < 1 || num_pages < 1)
+    return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: max_blocks and num_pages must be >= 1");
+  const long long cap = static_cast<long long>(max_blocks) * page_size;
+  if (cap > (1LL << 30)) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: capacity too large");
+  if (B > 0 && H > 0 && !block_table) return fail(FA_ERR_INVALID_ARG, "fa_decode_paged: null block_table");
+  int shift = 0;
+  while ((1 << shift) < page_size) ++shift;
+  return run_decode("fa_decode_paged", q, k_pages, v_pages, cache_seqlens, k_new, v_new, out, lse, B,
+                    H, static_cast<int>(cap), d, scale, block_table, max_blocks, shift, num_pages,
+                    stream);
 }
 
 fa_status fa_device_status(void* stream, unsigned int* site_out, unsigned int* info_out) {

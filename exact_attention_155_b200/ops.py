@@ -16,7 +16,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["FAError", "load_library", "fwd", "bwd", "fwd_ex", "bwd_ex", "fwd_qkvpacked",
-           "bwd_qkvpacked", "decode", "bwd_workspace_size", "decode_workspace_size",
+           "bwd_qkvpacked", "decode", "decode_paged", "bwd_workspace_size", "decode_workspace_size",
            "device_status", "debug_timeout_probe", "LIB_PATH", "declared_symbols"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -58,6 +58,9 @@ _SIGNATURES = {
     "fa_decode": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                            _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
                            _c_float, _c_void_p, _c_size_t, _c_void_p]),
+    "fa_decode_paged": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
+                                 _c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
+                                 _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p]),
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_device_status": (_c_int, [_c_void_p, ctypes.POINTER(ctypes.c_uint),
                                   ctypes.POINTER(ctypes.c_uint)]),
@@ -381,6 +384,46 @@ def decode(q, k_cache, v_cache, cache_seqlens, k_new=None, v_new=None, causal: b
                              _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(lse), B, H, Ncap, d,
                              int(bool(causal)), _scale(scale, d), _ptr(workspace), ws_bytes,
                              _stream(stream)))
+    return out, lse
+
+
+def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, k_new=None, v_new=None,
+                 causal: bool = True, scale: Optional[float] = None, out=None, lse=None,
+                 stream=None):
+    """One decode step over a paged cache (fa_decode_paged).
+
+    q: [B, 1, H, d]; k_pages, v_pages: [num_pages, page_size, H, d]; block_table: int32
+    [B, max_blocks] on the device; cache_seqlens: int32 [B] on the device. Returns
+    (out [B, 1, H, d] bf16, lse [B, H] fp32)."""
+    _require(q, "q")
+    _require(k_pages, "k_pages")
+    _require(v_pages, "v_pages")
+    _require(block_table, "block_table", torch.int32)
+    _require(cache_seqlens, "cache_seqlens", torch.int32)
+    B, one, H, d = q.shape
+    if one != 1 or k_pages.dim() != 4 or k_pages.shape != v_pages.shape \
+            or k_pages.shape[2] != H or k_pages.shape[3] != d:
+        raise ValueError("q must be [B,1,H,d] and pages [num_pages,page_size,H,d]")
+    if block_table.dim() != 2 or block_table.shape[0] != B:
+        raise ValueError("block_table must be int32 [B, max_blocks]")
+    if tuple(cache_seqlens.shape) != (B,):
+        raise ValueError("cache_seqlens must be int32 [B]")
+    num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new must be given together")
+    if k_new is not None:
+        _require(k_new, "k_new")
+        _require(v_new, "v_new")
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
+    _require(out, "out")
+    _require(lse, "lse", torch.float32)
+    lib = load_library()
+    with torch.cuda.device(q.device):
+        _check(lib.fa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                   block_table.shape[1], page_size, num_pages, _ptr(cache_seqlens),
+                                   _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(lse), B, H, d,
+                                   int(bool(causal)), _scale(scale, d), _stream(stream)))
     return out, lse
 
 

@@ -205,6 +205,26 @@ fa_status fa_decode(const void* q, void* k_cache, void* v_cache, const int* cach
                     int Ncap, int d, int causal, float scale, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/*
+ * The same decode step over a paged cache ("突破AI算力瓶颈：FlashAttention与MindSpore
+ * 2.0全场景融合方案": the KV cache of section 推理优化与KV缓存 is stored in pages to avoid
+ * fragmentation, and the paged cache is what its list of advantages credits for 100K+
+ * sequences): the caches are a pool of fixed-size pages shared by the batch,
+ *   k_pages, v_pages : [num_pages, page_size, H, d] bf16
+ *   block_table      : [B, max_blocks] int32 DEVICE array; row r of sequence b is row
+ *                      r % page_size of page block_table[b][r / page_size]
+ * page_size is a power of two; the logical capacity is max_blocks * page_size and
+ * plays the role of Ncap (a cache_seqlens value above it, or equal to it with k_new
+ * given, is FA_ERR_DEVICE_INPUT). The appended row goes to its page in place. A
+ * block-table entry that a row needs and that lies outside [0, num_pages) is recorded
+ * as FA_ERR_DEVICE_INPUT and that row is never read or written (it counts as masked).
+ * Other arguments, results and errors as fa_decode; no workspace is needed.
+ */
+fa_status fa_decode_paged(const void* q, void* k_pages, void* v_pages, const int* block_table,
+                          int max_blocks, int page_size, int num_pages, const int* cache_seqlens,
+                          const void* k_new, const void* v_new, void* out, float* lse, int B,
+                          int H, int d, int causal, float scale, void* stream);
+
 /* Message for the last non-OK status returned on the calling host thread. */
 const char* fa_last_error(void);
 
