@@ -509,6 +509,18 @@ def run_ours(args, rank, world, local_rank):
         vb_ms = timed_events(torch, bwd_v, 10)
         vf_fl = 4.0 * vb["d"] * vb["H"] * sum(n * (n + 1) // 2 for n in lens)
         del vq, vk, vv, vdo, vo, vlse, vg, vws
+        # Ring attention, 4 shards emulated on this GPU (exchange = indexing): the compute
+        # side of the sequence-parallel forward on the prefill workload.
+        from exact_attention_155_b200.ring import ring_attention_fwd_emulated
+        p = PREFILL
+        pin = attention_inputs(p["B"], p["N"], p["H"], p["d"], seed=1003, with_dout=False)
+        rq, rk, rv = (pin[n].to(dev) for n in ("q", "k", "v"))
+        del pin
+        ring_fn = lambda: ring_attention_fwd_emulated(rq, rk, rv, 4, causal=True, scale=scale)
+        for _ in range(2):
+            ring_fn()
+        rms = timed_events(torch, ring_fn, 5)
+        del rq, rk, rv
         parts = {
             "prefill_fwd": {"workload": "causal fwd B=1 H=32 N=8192 d=128", "value": ptf,
                             "unit": "TFLOP/s", "ms": pms, "roofline_bound": "tensor",
@@ -529,6 +541,12 @@ def run_ours(args, rank, world, local_rank):
                                    "peak": peaks["hbm"],
                                    "peak_kind": f"HBM copy, of {peaks['source']}",
                                    "l2": "flushed before every call"},
+            "ring_fwd_emulated": {
+                "workload": "causal fwd B=1 H=32 N=8192 d=128 as 4 sequence shards on one GPU "
+                            "(ring schedule, partial attention + LSE merge per shard pair)",
+                "value": fwd_flops(p["B"], p["H"], p["N"], p["d"], True) / (rms * 1e-3) / 1e12,
+                "unit": "TFLOP/s", "ms": rms,
+                "note": "exchange is indexing here; NCCL send/recv only with several GPUs"},
             "window_causal": {
                 "workload": f"causal sliding window {wwin[0]}, B=1 H=32 N=16384 d=128",
                 "fwd_tflops": wf_fl / (wf_ms * 1e-3) / 1e12, "fwd_ms": wf_ms,

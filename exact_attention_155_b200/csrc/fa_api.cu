@@ -17,6 +17,7 @@
 #include "fwd.cuh"
 #include "bwd.cuh"
 #include "decode.cuh"
+#include "merge.cuh"
 
 namespace {
 
@@ -675,6 +676,38 @@ fa_status fa_decode_paged(const void* q, void* k_pages, void* v_pages, const int
   return run_decode("fa_decode_paged", q, k_pages, v_pages, cache_seqlens, k_new, v_new, out, lse, B,
                     H, static_cast<int>(cap), d, scale, block_table, max_blocks, shift, num_pages,
                     stream);
+}
+
+fa_status fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                            void* out, int B, int N, int H, int d, void* stream) {
+  if (B < 0 || N < 0 || H < 0) return fail(FA_ERR_INVALID_ARG, "fa_merge_partials: negative size");
+  if (d != 64 && d != 128)
+    return fail(FA_ERR_UNSUPPORTED, "fa_merge_partials: head dim %d not supported (64 or 128)", d);
+  if (B == 0 || N == 0 || H == 0) return FA_OK;
+  if (!o_acc || !lse_acc || !o_part || !lse_part)
+    return fail(FA_ERR_INVALID_ARG, "fa_merge_partials: null pointer");
+  if (!aligned16(o_acc) || !aligned16(o_part) || !aligned4(lse_acc) || !aligned4(lse_part) ||
+      (out && !aligned16(out)))
+    return fail(FA_ERR_INVALID_ARG, "fa_merge_partials: o tensors 16-byte aligned, lse 4-byte");
+  const long long threads = static_cast<long long>(B) * N * H * (d / 8);
+  if (threads / 256 >= (1LL << 31)) return fail(FA_ERR_INVALID_ARG, "fa_merge_partials: too large");
+  int dev = 0;
+  fa_status st = current_device(&dev, nullptr);
+  if (st != FA_OK) return st;
+  fa::MergeParams p;
+  p.o_acc = o_acc;
+  p.lse_acc = lse_acc;
+  p.o_part = static_cast<const uint16_t*>(o_part);
+  p.lse_part = lse_part;
+  p.out = static_cast<uint16_t*>(out);
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64) fa::merge_kernel<64><<<blocks, 256, 0, s>>>(p);
+  else fa::merge_kernel<128><<<blocks, 256, 0, s>>>(p);
+  return check_launch("fa_merge_partials launch");
 }
 
 fa_status fa_device_status(void* stream, unsigned int* site_out, unsigned int* info_out) {

@@ -16,7 +16,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["FAError", "load_library", "fwd", "bwd", "fwd_ex", "bwd_ex", "fwd_qkvpacked",
-           "bwd_qkvpacked", "decode", "decode_paged", "bwd_workspace_size", "decode_workspace_size",
+           "bwd_qkvpacked", "decode", "decode_paged", "merge_partials", "bwd_workspace_size", "decode_workspace_size",
            "device_status", "debug_timeout_probe", "LIB_PATH", "declared_symbols"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -61,6 +61,8 @@ _SIGNATURES = {
     "fa_decode_paged": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int,
                                  _c_int, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                                  _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p]),
+    "fa_merge_partials": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int,
+                                   _c_int, _c_int, _c_int, _c_void_p]),
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_device_status": (_c_int, [_c_void_p, ctypes.POINTER(ctypes.c_uint),
                                   ctypes.POINTER(ctypes.c_uint)]),
@@ -425,6 +427,27 @@ def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, k_new=None, v_
                                    _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(lse), B, H, d,
                                    int(bool(causal)), _scale(scale, d), _stream(stream)))
     return out, lse
+
+
+def merge_partials(o_acc, lse_acc, o_part, lse_part, out=None, stream=None):
+    """Fold a partial result (o_part bf16 [B, N, H, d], lse_part [B, H, N]) into the
+    running one (o_acc fp32 [B, N, H, d], lse_acc [B, H, N]) in place (fa_merge_partials);
+    optionally write the merged output as bf16 into `out`."""
+    _require(o_acc, "o_acc", torch.float32)
+    _require(lse_acc, "lse_acc", torch.float32)
+    _require(o_part, "o_part")
+    _require(lse_part, "lse_part", torch.float32)
+    B, N, H, d = o_part.shape
+    if o_acc.shape != o_part.shape or tuple(lse_acc.shape) != (B, H, N) \
+            or tuple(lse_part.shape) != (B, H, N):
+        raise ValueError("o_acc/o_part must be [B, N, H, d] and lse_acc/lse_part [B, H, N]")
+    if out is not None:
+        _require(out, "out")
+    lib = load_library()
+    with torch.cuda.device(o_acc.device):
+        _check(lib.fa_merge_partials(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part),
+                                     _ptr(out), B, N, H, d, _stream(stream)))
+    return o_acc, lse_acc
 
 
 def device_status(stream=None):

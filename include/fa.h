@@ -229,6 +229,24 @@ fa_status fa_decode_paged(const void* q, void* k_pages, void* v_pages, const int
 const char* fa_last_error(void);
 
 /*
+ * Folds one partial attention result into a running one, for attention split over
+ * sequence shards (the ring sequence-parallel mode of "Flash-Attention 2/3在ms-swift中
+ * 的集成与性能提升", section on distributed training: each device attends its query
+ * shard to one key/value shard at a time and the results are combined). Both results
+ * are normalised over their own keys; the merge is the stable per-block combination of
+ * "FlashAttention优化Transformer显存与计算效率" section 2.2.2 in log space:
+ *   LSE = log(e^lse_acc + e^lse_part),
+ *   O   = e^(lse_acc - LSE) * O_acc + e^(lse_part - LSE) * O_part.
+ *   o_acc    : [B, N, H, d] fp32 (read, written)   lse_acc  : [B, H, N] fp32 (read, written)
+ *   o_part   : [B, N, H, d] bf16 (read)             lse_part : [B, H, N] fp32 (read)
+ *   out      : [B, N, H, d] bf16 copy of the merged output (written), or NULL
+ * Start from o_acc = 0 and lse_acc = -inf. A row where both LSEs are -inf keeps O_acc and
+ * -inf. Errors as fa_fwd.
+ */
+fa_status fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, const float* lse_part,
+                            void* out, int B, int N, int H, int d, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_DEVICE_INPUT or FA_ERR_CUDA.
  * If site_out / info_out are non-NULL they receive the reporting site id and an

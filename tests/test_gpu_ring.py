@@ -1,0 +1,60 @@
+"""Ring attention pieces on one GPU: the LSE merge kernel against the oracle's merge,
+and the full ring schedule for 1, 2 and 4 shards emulated in one process (the shard
+exchange becomes indexing) against the oracle's attention over the whole sequence."""
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_155_b200 as fa
+import oracle
+from exact_attention_155_b200.inputs import bf16_randn, to_f64
+from exact_attention_155_b200.ring import ring_attention_fwd_emulated
+from helpers import LSE_ATOL, OUT_ATOL, check_fwd, default_scale, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_merge_kernel_matches_oracle_merge(d):
+    B, N, H = 2, 77, 3
+    g = torch.Generator().manual_seed(9970 + d)
+    o1 = torch.randn((B, N, H, d), generator=g, dtype=torch.float32)
+    o2 = bf16_randn((B, N, H, d), g)
+    l1 = torch.randn((B, H, N), generator=g) * 3
+    l2 = torch.randn((B, H, N), generator=g) * 3
+    l1[0, 0, :5] = float("-inf")   # nothing merged yet on some rows
+    l2[1, 2, 3:9] = float("-inf")  # an empty partial on others
+    l1[1, 1, 10] = l2[1, 1, 10] = float("-inf")  # both empty
+    o_acc, lse_acc = o1.cuda(), l1.cuda()
+    out = torch.empty((B, N, H, d), dtype=torch.bfloat16, device="cuda")
+    fa.ops.merge_partials(o_acc, lse_acc, o2.cuda(), l2.cuda(), out=out)
+    torch.cuda.synchronize()
+    # The oracle takes each LSE in the layout of its output rows: [B, N, H].
+    ref_o, ref_l = oracle.merge_partials(
+        np.stack([o1.numpy().astype(np.float64), to_f64(o2)]),
+        np.stack([l1.numpy().transpose(0, 2, 1), l2.numpy().transpose(0, 2, 1)]).astype(np.float64))
+    ref_l = ref_l.transpose(0, 2, 1)  # back to [B, H, N]
+    both_empty = np.isneginf(l1.numpy()) & np.isneginf(l2.numpy())
+    # Where both parts are empty the running output is kept (the oracle returns 0).
+    keep = np.repeat(both_empty.transpose(0, 2, 1)[..., None], d, axis=-1)
+    ref_o = np.where(keep, o1.numpy(), ref_o)
+    got_o = o_acc.cpu().numpy()
+    assert np.max(np.abs(got_o - ref_o)) <= 1e-5 * max(1.0, np.max(np.abs(ref_o)))
+    got_l = lse_acc.cpu().numpy()
+    fin = np.isfinite(ref_l)
+    assert np.array_equal(np.isneginf(got_l), np.isneginf(ref_l))
+    assert np.max(np.abs(got_l[fin] - ref_l[fin])) <= 1e-5
+    assert torch.equal(out, o_acc.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("world", [1, 2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_emulated_ring_matches_whole_sequence(world, causal, d):
+    B, N, H = 1, 1024, 2
+    inp = make_inputs(B, N, H, d, 9980 + world + d + int(causal), with_dout=False)
+    q, k, v = (inp[n].cuda() for n in ("q", "k", "v"))
+    sc = default_scale(d)
+    out, lse = ring_attention_fwd_emulated(q, k, v, world, causal=causal, scale=sc)
+    torch.cuda.synchronize()
+    check_fwd(out, lse, inp, causal, sc)
