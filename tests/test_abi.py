@@ -126,6 +126,30 @@ def test_bwd_ex_argument_errors(lib):
     assert call(ws=NULL) == WORKSPACE
 
 
+def test_decode_paged_argument_errors(lib):
+    def call(page_size=64, max_blocks=4, num_pages=8, table=P16, d=64, B=2, kn=NULL, vn=NULL):
+        return lib.fa_decode_paged(P16, P16, P16, table, max_blocks, page_size, num_pages, P16, kn, vn,
+                                   P16, NULL, B, 2, d, 1, 0.125, NULL)
+    assert call(page_size=48) == INVALID  # not a power of two
+    assert b"power of two" in lib.fa_last_error()
+    assert call(page_size=0) == INVALID
+    assert call(max_blocks=0) == INVALID
+    assert call(num_pages=0) == INVALID
+    assert call(table=NULL) == INVALID
+    assert call(kn=P16) == INVALID  # k_new without v_new
+    assert call(d=96) == UNSUPPORTED
+    assert call(B=0) == FA_OK
+
+
+def test_merge_partials_argument_errors(lib):
+    def call(o=P16, l=P16, op=P16, lp=P16, out=NULL, d=64, N=8):
+        return lib.fa_merge_partials(o, l, op, lp, out, 1, N, 2, d, NULL)
+    assert call(d=80) == UNSUPPORTED
+    assert call(o=NULL) == INVALID
+    assert call(out=P_ODD) == INVALID
+    assert call(N=0) == FA_OK
+
+
 def _dec(lib, q=P16, kn=NULL, vn=NULL, seq=P16, Ncap=2048, d=64, B=2):
     return lib.fa_decode(q, P16, P16, seq, kn, vn, P16, NULL, B, 16, Ncap, d, 1, 0.125, NULL, 0, S0)
 
