@@ -47,8 +47,8 @@ STEPS5 = dict(B=2, H=16, d=64, Ncap=2048, steps=100)
 
 # DRAM bytes per launch of the backward main kernel from an ncu capture, valid only
 # for the kernel source it was taken on (sha256 of csrc/bwd.cuh).
-BWD_TRAFFIC = {"src_sha256": "4d16e5b0a9ca117874aba48e32804f1f24e8d04b97f2a5ed4e4e9b65e808269d",
-               "bytes_per_launch": 830.93e6 + 511.71e6,
+BWD_TRAFFIC = {"src_sha256": "162d783fc1a81100ca0bae73729dc9b95f88603fc6710fc936be1b3b05a67208",
+               "bytes_per_launch": 828.82e6 + 509.35e6,
                "profile": "profiles/bwd_kernel_train_causal_B1_H32_N16384_d128.md"}
 
 
