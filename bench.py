@@ -47,6 +47,10 @@ STEPS5 = dict(B=2, H=16, d=64, Ncap=2048, steps=100)
 
 # DRAM bytes per launch of the backward main kernel from an ncu capture, valid only
 # for the kernel source it was taken on (sha256 of csrc/bwd.cuh).
+# Throughput of cp.reduce.async.bulk .add.f32 from shared memory into a 256 MiB fp32
+# buffer, all SMs reducing 16 KB chunks (independent of 2, 4 or 8 chunks in flight per SM).
+L2_REDUCTION_GBS = 3840.0
+
 BWD_TRAFFIC = {"src_sha256": "162d783fc1a81100ca0bae73729dc9b95f88603fc6710fc936be1b3b05a67208",
                "bytes_per_launch": 828.82e6 + 509.35e6,
                "profile": "profiles/bwd_kernel_train_causal_B1_H32_N16384_d128.md"}
@@ -318,6 +322,18 @@ def run_ours(args, rank, world, local_rank):
                 "peak_kind": f"bf16 dense, sustained, of {peaks['source']}",
                 "traffic": traffic, "avg_launch_ms": bwd_main_ms,
                 "algorithmic_flop_per_launch": f_bwd}
+    # The backward's other bound: every (key tile, visible query tile) pair adds a
+    # 128 x d fp32 block of dQ into the L2-resident accumulator with a bulk reduction.
+    nkt = (w["N"] + 127) // 128
+    pairs = nkt * (nkt + 1) // 2 if w["causal"] else nkt * nkt
+    red_bytes = float(pairs) * 128 * w["d"] * 4 * w["B"] * w["H"]
+    roofline["l2_reduction"] = {
+        "bytes_per_launch": red_bytes,
+        "achieved_gbs": red_bytes / (bwd_main_ms * 1e-3) / 1e9,
+        "peak_gbs": L2_REDUCTION_GBS,
+        "frac": red_bytes / (bwd_main_ms * 1e-3) / 1e9 / L2_REDUCTION_GBS,
+        "peak_kind": "bulk fp32 reductions into L2, 148 CTAs, measured by a microbenchmark "
+                     "(not in the driver's peak file)"}
 
     # ---- end to end through the public API from pinned host buffers
     # Every step copies its own inputs host->device and its results device->host.
