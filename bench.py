@@ -48,7 +48,8 @@ STEPS5 = dict(B=2, H=16, d=64, Ncap=2048, steps=100)
 # DRAM bytes per launch of the backward main kernel from an ncu capture, valid only
 # for the kernel source it was taken on (sha256 of csrc/bwd.cuh).
 # Throughput of cp.reduce.async.bulk .add.f32 from shared memory into a 256 MiB fp32
-# buffer, all SMs reducing 16 KB chunks (independent of 2, 4 or 8 chunks in flight per SM).
+# buffer, all SMs reducing 16 KB chunks (independent of 2, 4 or 8 chunks in flight per SM),
+# measured on this machine type by exact_attention_155_b200/csrc/l2_reduction_rate.cu.
 L2_REDUCTION_GBS = 3840.0
 
 BWD_TRAFFIC = {"src_sha256": "162d783fc1a81100ca0bae73729dc9b95f88603fc6710fc936be1b3b05a67208",
