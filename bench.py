@@ -52,7 +52,7 @@ STEPS5 = dict(B=2, H=16, d=64, Ncap=2048, steps=100)
 # measured on this machine type by exact_attention_155_b200/csrc/l2_reduction_rate.cu.
 L2_REDUCTION_GBS = 3840.0
 
-BWD_TRAFFIC = {"src_sha256": "162d783fc1a81100ca0bae73729dc9b95f88603fc6710fc936be1b3b05a67208",
+BWD_TRAFFIC = {"src_sha256": "00ade1531fe1e214ba9fdbe8ae5ee1f1bf2a53490bebce85486bcab486fb1ad7",
                "bytes_per_launch": 828.82e6 + 509.35e6,
                "profile": "profiles/bwd_kernel_train_causal_B1_H32_N16384_d128.md"}
 

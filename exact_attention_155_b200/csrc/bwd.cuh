@@ -475,7 +475,7 @@ __global__ void __launch_bounds__(448, 1)
     const bool key_ok = key < seqlen;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float sl2 = p.scale_log2;
-    const bool tr = blockIdx.x == 0 && threadIdx.x == 0;
+    [[maybe_unused]] const bool tr = blockIdx.x == 0 && threadIdx.x == 0;  // traced thread
     bool ok = true;
     for (int n = 0; n < niter; ++n) {
       const int it = it0 + n;

@@ -89,17 +89,6 @@ fa_status current_device(int* dev_out, int* sms_out) {
   return FA_OK;
 }
 
-// SM count used for sizing decisions that must also be answerable without a GPU
-// (workspace queries): the current device's count when there is one, else 148.
-int sm_count_or_default() {
-  int dev = 0, sms = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess &&
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && sms > 0)
-    return sms;
-  cudaGetLastError();  // clear the "no device" error so it does not leak into later calls
-  return 148;
-}
-
 // ------------------------------------------------------------- TMA descriptors
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,

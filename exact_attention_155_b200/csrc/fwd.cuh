@@ -414,7 +414,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const float sl2 = p.scale_log2;
     float* xmax = reinterpret_cast<float*>(smem + L::kXMaxOff);
     float* xsum = reinterpret_cast<float*>(smem + L::kXSumOff);
-    const bool tr = blockIdx.x == 0 && grp == 0 && lane == 0;  // group 0, one thread per warp
+    [[maybe_unused]] const bool tr = blockIdx.x == 0 && grp == 0 && lane == 0;  // traced threads
     float m[2] = {-INFINITY, -INFINITY};  // running row max per tile (log2 units)
     float l[2] = {0.f, 0.f};              // running exp-sum over this group's columns
     bool ok = true;
