@@ -23,7 +23,7 @@
 //    (tile 0, then tile 1, per key tile), so all of them keep the exponential unit
 //    busy while the tensor pipe computes the other tile's products; exponentials are
 //    computed against the current reference max and redone only in the rare steps
-//    where a row grew past it; P is published to the MMA warp per 64-key half;
+//    where a row grew past it; P is published to the tile's MMA warp per 64-key half;
 //  * TMEM columns: S_0 [0,128) S_1 [128,256) O_0 [256,256+d) O_1 [256+d,256+2d).
 #pragma once
 
@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // The softmax warps work on one Q tile at a time (tile 0, then tile 1, for every
     // key tile j). Group g (warps 4g..4g+3) takes key columns [g*C, g*C + C),
     // C = 128 / kFwdGroups, of each of the 128 rows (one TMEM lane per row), so all
-    // softmax warps share the exponential unit on one tile while the MMA warp runs
+    // softmax warps share the exponential unit on one tile while the tensor pipe runs
     // the other tile's products. Column groups of a row meet in shared memory only
     // on exact steps (row maxima) and at the end (exp-sums).
     constexpr int C = kFwdCols;
