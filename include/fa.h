@@ -15,13 +15,16 @@
  *    gradients are bf16 (passed as void*, 2 bytes per element) in the layout
  *    [B, N, H, d] = (batch, seq_len, heads, head_dim), the layout of section 1.1 of
  *    "ms-swift长文本训练优化，Flash-Attention显存省一半". Every bf16 pointer must be
- *    16-byte aligned; float pointers 4-byte aligned.
+ *    16-byte aligned; float pointers 4-byte aligned. (fa_fwd_ex / fa_bwd_ex also take
+ *    row strides and packed variable-length batches, fa_decode_paged a paged cache;
+ *    their comments give the layouts.)
  *  - d (head_dim) must be 64 or 128. The device must be compute capability 10.0
  *    (B200, sm_100a).
  *  - scale is the softmax scale; any finite value. (The pages' softmax_scale=None
  *    default, 1/sqrt(d), is applied by the Python binding, not here.)
  *  - LSE is the natural-log log-sum-exp of each query row's scaled scores over its
- *    visible keys, fp32, laid out [B, H, N]. A row with no visible key gets -inf.
+ *    visible keys, fp32, laid out [B, H, N] ([H, total] for a packed variable-length
+ *    call). A row with no visible key gets -inf.
  *  - causal != 0 masks key j for query i when j > i (for decode, the single new
  *    query sees every valid key, so causal changes nothing there).
  *  - stream is a cudaStream_t (NULL = legacy default stream). Every call only
