@@ -47,6 +47,11 @@ STEPS5 = dict(B=2, H=16, d=64, Ncap=2048, steps=100)
 
 # DRAM bytes per launch of the backward main kernel from an ncu capture, valid only
 # for the kernel source it was taken on (sha256 of csrc/bwd.cuh).
+# Nominal B200 figures the targets are stated against (dense bf16, HBM3e): reported
+# beside the measured-peak fractions.
+NOMINAL_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 8000.0
+
 # Throughput of cp.reduce.async.bulk .add.f32 from shared memory into a 256 MiB fp32
 # buffer, all SMs reducing 16 KB chunks (independent of 2, 4 or 8 chunks in flight per SM),
 # measured on this machine type by exact_attention_155_b200/csrc/l2_reduction_rate.cu.
@@ -320,6 +325,7 @@ def run_ours(args, rank, world, local_rank):
     roofline = {"kernel": "bwd_kernel<128,causal>", "bound": "tensor", "achieved": achieved,
                 "peak": peaks["tf_sustained"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["tf_sustained"],
+                "frac_of_nominal": achieved / NOMINAL_TFLOPS,
                 "peak_kind": f"bf16 dense, sustained, of {peaks['source']}",
                 "traffic": traffic, "avg_launch_ms": bwd_main_ms,
                 "algorithmic_flop_per_launch": f_bwd}
@@ -542,6 +548,7 @@ def run_ours(args, rank, world, local_rank):
             "prefill_fwd": {"workload": "causal fwd B=1 H=32 N=8192 d=128", "value": ptf,
                             "unit": "TFLOP/s", "ms": pms, "roofline_bound": "tensor",
                             "frac": ptf / peaks["tf_burst"],
+                            "frac_of_nominal": ptf / NOMINAL_TFLOPS,
                             "peak": peaks["tf_burst"],
                             "peak_kind": f"bf16 dense, burst, of {peaks['source']}"},
             "train_fwd_in_step": {"value": f_fwd / (fwd_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -549,6 +556,7 @@ def run_ours(args, rank, world, local_rank):
             "decode_sweep": {"workload": "decode B=32 H=16 d=64, 2048 cached rows, no append",
                              "value": dgbs, "unit": "GB/s", "us": dms * 1e3,
                              "roofline_bound": "hbm", "frac": dgbs / peaks["hbm"],
+                             "frac_of_nominal": dgbs / NOMINAL_HBM_GBS,
                              "peak": peaks["hbm"], "peak_kind": f"HBM copy, of {peaks['source']}",
                              "l2": "flushed before every call (512 MiB write, then 256 MiB read)"},
             "decode_sweep_paged": {"workload": "decode B=32 H=16 d=64, 2048 rows in 64-row pages "
