@@ -18,6 +18,7 @@
 #include "bwd.cuh"
 #include "decode.cuh"
 #include "merge.cuh"
+#include "accumulate.cuh"
 
 namespace {
 
@@ -697,6 +698,28 @@ fa_status fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, co
   if (d == 64) fa::merge_kernel<64><<<blocks, 256, 0, s>>>(p);
   else fa::merge_kernel<128><<<blocks, 256, 0, s>>>(p);
   return check_launch("fa_merge_partials launch");
+}
+
+fa_status fa_accumulate(float* acc, const void* part, void* out, long long n, void* stream) {
+  if (n < 0) return fail(FA_ERR_INVALID_ARG, "fa_accumulate: n < 0");
+  if (n == 0) return FA_OK;
+  if (!acc) return fail(FA_ERR_INVALID_ARG, "fa_accumulate: null acc");
+  if (!part && !out) return fail(FA_ERR_INVALID_ARG, "fa_accumulate: part and out are both NULL");
+  if (n % 8 != 0) return fail(FA_ERR_INVALID_ARG, "fa_accumulate: n (%lld) must be a multiple of 8", n);
+  if (!aligned16(acc) || (part && !aligned16(part)) || (out && !aligned16(out)))
+    return fail(FA_ERR_INVALID_ARG, "fa_accumulate: acc, part and out must be 16-byte aligned");
+  const long long n8 = n / 8;
+  const long long blocks = (n8 + 255) / 256;
+  if (blocks >= (1LL << 31)) return fail(FA_ERR_INVALID_ARG, "fa_accumulate: n too large");
+  fa_status st = current_device(nullptr, nullptr);
+  if (st != FA_OK) return st;
+  fa::AccumParams p;
+  p.acc = acc;
+  p.part = static_cast<const uint16_t*>(part);
+  p.out = static_cast<uint16_t*>(out);
+  p.n8 = n8;
+  fa::accumulate_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(p);
+  return check_launch("fa_accumulate launch");
 }
 
 fa_status fa_device_status(void* stream, unsigned int* site_out, unsigned int* info_out) {

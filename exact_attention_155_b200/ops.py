@@ -16,7 +16,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["FAError", "load_library", "fwd", "bwd", "fwd_ex", "bwd_ex", "fwd_qkvpacked",
-           "bwd_qkvpacked", "decode", "decode_paged", "merge_partials", "bwd_workspace_size", "decode_workspace_size",
+           "bwd_qkvpacked", "decode", "decode_paged", "merge_partials", "accumulate", "bwd_workspace_size", "decode_workspace_size",
            "device_status", "debug_timeout_probe", "LIB_PATH", "declared_symbols"]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa.so")
@@ -63,6 +63,7 @@ _SIGNATURES = {
                                  _c_int, _c_int, _c_int, _c_int, _c_float, _c_void_p]),
     "fa_merge_partials": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int,
                                    _c_int, _c_int, _c_int, _c_void_p]),
+    "fa_accumulate": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_ll, _c_void_p]),
     "fa_last_error": (ctypes.c_char_p, []),
     "fa_device_status": (_c_int, [_c_void_p, ctypes.POINTER(ctypes.c_uint),
                                   ctypes.POINTER(ctypes.c_uint)]),
@@ -448,6 +449,23 @@ def merge_partials(o_acc, lse_acc, o_part, lse_part, out=None, stream=None):
         _check(lib.fa_merge_partials(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part),
                                      _ptr(out), B, N, H, d, _stream(stream)))
     return o_acc, lse_acc
+
+
+def accumulate(acc, part=None, out=None, stream=None):
+    """acc (fp32) += part (bf16, same shape) in place when part is given, then write the
+    sum as bf16 into `out` when given (fa_accumulate). Returns acc."""
+    _require(acc, "acc", torch.float32)
+    if part is None and out is None:
+        raise ValueError("give part, out or both")
+    for name, t in (("part", part), ("out", out)):
+        if t is not None:
+            _require(t, name)
+            if t.shape != acc.shape or t.device != acc.device:
+                raise ValueError(f"{name} must have acc's shape and device")
+    lib = load_library()
+    with torch.cuda.device(acc.device):
+        _check(lib.fa_accumulate(_ptr(acc), _ptr(part), _ptr(out), acc.numel(), _stream(stream)))
+    return acc
 
 
 def device_status(stream=None):

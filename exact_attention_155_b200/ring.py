@@ -8,9 +8,16 @@ Rank r holds rows [r*S, (r+1)*S) of q, k and v (S = N / world). At step s it hol
 the key/value shard of rank (r - s) mod world, attends its query shard to it with
 fa_fwd_ex (causal only on its own shard; shards after its own are skipped when
 causal), folds the partial result into a running fp32 output with fa_merge_partials,
-and passes the shard on to rank r + 1 while it computes. Every arithmetic step runs in
-the CUDA library; this module only orders calls and moves buffers (torch.distributed
-point-to-point, NCCL on GPUs).
+and passes the shard on to rank r + 1 while it computes.
+
+The backward visits the shards in the same order. With the forward's output and LSE of
+its query rows fixed, the recomputed backward of one (query shard, key/value shard)
+pair (fa_bwd_ex) gives that pair's terms of dQ, dK and dV, and each gradient is the sum
+of its terms (fa_accumulate keeps the sums in fp32). dQ stays on its rank; the sums
+for dK and dV travel with their key/value shard and reach its owner after a full turn.
+
+Every arithmetic step runs in the CUDA library; this module only orders calls and
+moves buffers (torch.distributed point-to-point, NCCL on GPUs).
 """
 from __future__ import annotations
 
@@ -49,19 +56,44 @@ def ring_pass(send: torch.Tensor, recv: torch.Tensor, rank: int, world: int, gro
     return dist.batch_isend_irecv(ops_)
 
 
+def last_step(schedule) -> int:
+    """The last step of a schedule that is not skipped (a rank always attends its own
+    shard, at step 0): the step whose merge or sum also writes the bf16 result."""
+    return max(s for s, _, mode in schedule if mode != SKIP)
+
+
 def _attend_and_merge(q, k, v, mode, scale, o_acc, lse_acc, out, stream=None):
+    """Folds the attention of q to one key/value shard into (o_acc, lse_acc); writes
+    the merged output as bf16 into `out` when given."""
     if mode == SKIP:
         return
     o_p, lse_p = ops.fwd_ex(q, k, v, causal=(mode == CAUSAL), scale=scale, stream=stream)
     ops.merge_partials(o_acc, lse_acc, o_p, lse_p, out=out, stream=stream)
 
 
-def _finish(o_acc, out):
-    # Rows whose every shard was skipped cannot occur (a rank always attends its own
-    # shard); the last merge wrote `out` unless the last steps were skipped, so write
-    # it from the accumulator here in every case.
-    out.copy_(o_acc.to(torch.bfloat16))
-    return out
+def _grad_terms(q, k, v, out, dout, lse, mode, scale, dq_acc, dk_acc, dv_acc, dq_out, bufs,
+                stream=None):
+    """Adds the terms of one (query shard, key/value shard) pair to the fp32 sums
+    dq_acc, dk_acc, dv_acc; writes the dQ sum as bf16 into `dq_out` when given. `bufs`
+    holds the bf16 term buffers and the backward workspace, made on first use."""
+    if mode == SKIP:
+        return
+    if not bufs:
+        B, S, H, d = q.shape
+        bufs["terms"] = tuple(torch.empty_like(q) for _ in range(3))
+        bufs["ws"] = torch.empty(max(1, ops.bwd_workspace_size(B, H, S, d)), dtype=torch.uint8,
+                                 device=q.device)
+    tq, tk, tv = bufs["terms"]
+    ops.bwd_ex(q, k, v, out, dout, lse, causal=(mode == CAUSAL), scale=scale, dq=tq, dk=tk, dv=tv,
+               workspace=bufs["ws"], stream=stream)
+    ops.accumulate(dq_acc, tq, out=dq_out, stream=stream)
+    ops.accumulate(dk_acc, tk, stream=stream)
+    ops.accumulate(dv_acc, tv, stream=stream)
+
+
+def _to_bf16(acc, out, stream=None):
+    """Writes the fp32 sum `acc` as bf16 into `out`."""
+    ops.accumulate(acc, None, out=out, stream=stream)
 
 
 def ring_attention_fwd(q, k, v, causal: bool = False, scale: Optional[float] = None, group=None):
@@ -76,13 +108,15 @@ def ring_attention_fwd(q, k, v, causal: bool = False, scale: Optional[float] = N
     o_acc = torch.zeros((B, S, H, d), dtype=torch.float32, device=q.device)
     lse_acc = torch.full((B, H, S), float("-inf"), dtype=torch.float32, device=q.device)
     out = torch.empty_like(q)
-    for s, src, mode in ring_schedule(rank, world, causal):
+    sched = ring_schedule(rank, world, causal)
+    last = last_step(sched)
+    for s, src, mode in sched:
         reqs = ring_pass(kv, nxt, rank, world, group) if s + 1 < world else []
-        _attend_and_merge(q, kv[0], kv[1], mode, scale, o_acc, lse_acc, None)
+        _attend_and_merge(q, kv[0], kv[1], mode, scale, o_acc, lse_acc, out if s == last else None)
         for r in reqs:
             r.wait()
         kv, nxt = nxt, kv
-    return _finish(o_acc, out), lse_acc
+    return out, lse_acc
 
 
 def ring_attention_fwd_emulated(q, k, v, world: int, causal: bool = False,
@@ -99,10 +133,86 @@ def ring_attention_fwd_emulated(q, k, v, world: int, causal: bool = False,
         qs = q[:, rank * S:(rank + 1) * S].contiguous()
         o_acc = torch.zeros((B, S, H, d), dtype=torch.float32, device=q.device)
         lse_acc = torch.full((B, H, S), float("-inf"), dtype=torch.float32, device=q.device)
-        for _, src, mode in ring_schedule(rank, world, causal):
+        out = torch.empty_like(qs)
+        sched = ring_schedule(rank, world, causal)
+        last = last_step(sched)
+        for s, src, mode in sched:
             ks = k[:, src * S:(src + 1) * S].contiguous()
             vs = v[:, src * S:(src + 1) * S].contiguous()
-            _attend_and_merge(qs, ks, vs, mode, scale, o_acc, lse_acc, None)
-        outs.append(_finish(o_acc, torch.empty_like(qs)))
+            _attend_and_merge(qs, ks, vs, mode, scale, o_acc, lse_acc, out if s == last else None)
+        outs.append(out)
         lses.append(lse_acc)
     return torch.cat(outs, dim=1), torch.cat(lses, dim=2)
+
+
+def ring_attention_bwd(q, k, v, out, dout, lse, causal: bool = False,
+                       scale: Optional[float] = None, group=None):
+    """Distributed backward of ring_attention_fwd. q, k, v, out, dout: this rank's
+    shards [B, S, H, d] bf16 (out as ring_attention_fwd returned it); lse: this rank's
+    rows of the LSE over the whole sequence [B, H, S] fp32. Returns (dq, dk, dv) of this
+    rank's shards, bf16."""
+    import torch.distributed as dist
+    rank, world = dist.get_rank(group), dist.get_world_size(group)
+    kv = torch.stack([k, v]).contiguous()
+    nxt = torch.empty_like(kv)
+    dkv = torch.zeros((2, *q.shape), dtype=torch.float32, device=q.device)
+    dkv_nxt = torch.empty_like(dkv)
+    dq_acc = torch.zeros(q.shape, dtype=torch.float32, device=q.device)
+    dq = torch.empty_like(q)
+    sched = ring_schedule(rank, world, causal)
+    last = last_step(sched)
+    bufs = {}
+    for s, src, mode in sched:
+        reqs = ring_pass(kv, nxt, rank, world, group) if s + 1 < world else []
+        _grad_terms(q, kv[0], kv[1], out, dout, lse, mode, scale, dq_acc, dkv[0], dkv[1],
+                    dq if s == last else None, bufs)
+        for r in reqs:
+            r.wait()
+        if world > 1:
+            # The dK/dV sums of the shard held now move on with it; after the last step
+            # this pass brings every rank the sums of its own shard.
+            for r in ring_pass(dkv, dkv_nxt, rank, world, group):
+                r.wait()
+            dkv, dkv_nxt = dkv_nxt, dkv
+        kv, nxt = nxt, kv
+    dk, dv = torch.empty_like(k), torch.empty_like(v)
+    _to_bf16(dkv[0], dk)
+    _to_bf16(dkv[1], dv)
+    return dq, dk, dv
+
+
+def ring_attention_bwd_emulated(q, k, v, out, dout, lse, world: int, causal: bool = False,
+                                scale: Optional[float] = None):
+    """ring_attention_bwd's schedule and kernels for `world` virtual ranks in one
+    process on one GPU (the travelling dK/dV sums become one sum per shard); q, k, v,
+    out, dout are the whole [B, N, H, d] tensors and lse [B, H, N]. Returns (dq, dk, dv)
+    [B, N, H, d]."""
+    B, N, H, d = q.shape
+    if N % world:
+        raise ValueError("N must be a multiple of the number of shards")
+    S = N // world
+    rows = lambda t, r: t[:, r * S:(r + 1) * S].contiguous()
+    ks = [rows(k, r) for r in range(world)]
+    vs = [rows(v, r) for r in range(world)]
+    dk_acc = [torch.zeros((B, S, H, d), dtype=torch.float32, device=q.device) for _ in range(world)]
+    dv_acc = [torch.zeros((B, S, H, d), dtype=torch.float32, device=q.device) for _ in range(world)]
+    bufs = {}
+    dqs = []
+    for rank in range(world):
+        qs, os_, dos = rows(q, rank), rows(out, rank), rows(dout, rank)
+        ls = lse[:, :, rank * S:(rank + 1) * S].contiguous()
+        dq_acc = torch.zeros((B, S, H, d), dtype=torch.float32, device=q.device)
+        dq = torch.empty_like(qs)
+        sched = ring_schedule(rank, world, causal)
+        last = last_step(sched)
+        for s, src, mode in sched:
+            _grad_terms(qs, ks[src], vs[src], os_, dos, ls, mode, scale, dq_acc, dk_acc[src],
+                        dv_acc[src], dq if s == last else None, bufs)
+        dqs.append(dq)
+    dks, dvs = [], []
+    for j in range(world):
+        dks.append(torch.empty_like(ks[j]))
+        dvs.append(torch.empty_like(vs[j]))
+        _to_bf16(dk_acc[j], dks[j])
+        _to_bf16(dv_acc[j], dvs[j])
+    return torch.cat(dqs, dim=1), torch.cat(dks, dim=1), torch.cat(dvs, dim=1)

@@ -250,6 +250,25 @@ fa_status fa_merge_partials(float* o_acc, float* lse_acc, const void* o_part, co
                             void* out, int B, int N, int H, int d, void* stream);
 
 /*
+ * Running fp32 sum of bf16 partial results, for the backward of attention split over
+ * sequence shards (the ring sequence-parallel mode of "Flash-Attention 2/3在ms-swift中
+ * 的集成与性能提升", section on distributed training). With the forward's LSE and output
+ * of every query row given, the recomputed backward ("ms-swift长文本训练优化，Flash-
+ * Attention显存省一半" section 1.2) of one query shard against one key/value shard
+ * (fa_bwd_ex) yields that pair's terms of dQ, dK and dV; each gradient is the sum of
+ * its terms over the other operand's shards.
+ *   acc  : n fp32 (read, written)      acc[i] += (float)part[i]  when part != NULL
+ *   part : n bf16 (read), or NULL
+ *   out  : n bf16 (written), or NULL   out[i] = bf16_rne(acc[i]) after the addition
+ * At least one of part and out is non-NULL; n >= 0 is a multiple of 8 (n = 0 is a
+ * no-op); all three pointers are 16-byte aligned device memory, any layout (the
+ * operation is elementwise). Errors: FA_ERR_INVALID_ARG for a bad n, pointer or
+ * alignment, before any launch; FA_ERR_UNSUPPORTED off sm_100; FA_ERR_CUDA for a
+ * launch error.
+ */
+fa_status fa_accumulate(float* acc, const void* part, void* out, long long n, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the device status word of the
  * current device. Returns FA_OK, FA_ERR_TIMEOUT, FA_ERR_DEVICE_INPUT or FA_ERR_CUDA.
  * If site_out / info_out are non-NULL they receive the reporting site id and an

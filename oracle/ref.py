@@ -50,6 +50,10 @@ Readings taken where the pages are silent (each is also listed in the design not
   sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]); each sequence is an
   independent attention problem (nothing is attended across sequences); the LSE is
   laid out [H, total].
+* Ring attention's backward ("Flash-Attention 2/3在ms-swift中的集成与性能提升", section on
+  distributed training, names the ring for training but gives no backward): with each
+  query row's LSE and output taken from the whole sequence, the backward's terms for one
+  key shard add up over the shards to the gradients (attention_backward_from_stats).
 
 Every array is numpy float64; callers convert the exact bf16 input values first.
 Large problems are processed in blocks of query rows; each block's softmax is the
@@ -70,6 +74,7 @@ __all__ = [
     "softmax_rows",
     "attention_forward",
     "attention_backward",
+    "attention_backward_from_stats",
     "attention_forward_varlen",
     "attention_backward_varlen",
     "blockwise_forward",
@@ -219,6 +224,52 @@ def attention_backward(q, k, v, dout, causal=False, scale=None, row_block=1024,
             dk_acc += sc * (ds.T @ qm)
         dk[b, :, h, :] = dk_acc
         dv[b, :, h, :] = dv_acc
+    return dq, dk, dv
+
+
+def attention_backward_from_stats(q, k, v, out, dout, lse, causal=False, scale=None):
+    """The backward's terms for one key set, with the softmax statistics of every query
+    row given rather than computed over these keys.
+
+    The backward recomputes the probabilities from Q, K and what the forward kept
+    (the recomputation of the ms-swift FA2/3 page's key-techniques list and section 1.2
+    of "ms-swift长文本训练优化，Flash-Attention显存省一半"): P = exp(scale*Q K^T - lse)
+    on visible entries, with lse the row's log-sum-exp over ALL its keys, and the
+    row term rowsum(P * dP) of the softmax gradient written as rowsum(dO * O) with O
+    the row's full output (the two are equal when the key set is complete). Then
+      dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),  dQ = scale dS K,
+      dK = scale dS^T Q.
+    Over a partition of the keys the terms add up to attention_backward's gradients;
+    this is how attention split over sequence shards gets its gradients.
+
+    q, out, dout: [B, Nq, H, d]; k, v: [B, Nk, H, d]; lse: [B, H, Nq]. Returns the
+    terms dq [B, Nq, H, d], dk, dv [B, Nk, H, d].
+    """
+    q, k, v, out, dout, lse = (np.asarray(t, dtype=np.float64) for t in (q, k, v, out, dout, lse))
+    B, Nq, H, d = q.shape
+    Nk = k.shape[1]
+    sc = _resolve_scale(scale, d)
+    dq = np.zeros(q.shape)
+    dk = np.zeros(k.shape)
+    dv = np.zeros(v.shape)
+    ridx = np.arange(Nq)
+    mask = _mask(ridx, Nk, causal, Nq, -1, -1)
+    for b in range(B):
+        for h in range(H):
+            qm, km, vm = q[b, :, h, :], k[b, :, h, :], v[b, :, h, :]
+            dom = dout[b, :, h, :]
+            row_lse = lse[b, h, :][:, None]
+            fin = np.isfinite(row_lse)  # lse = -inf: the row sees no key at all
+            live = mask & fin
+            shifted = scores(qm, km, sc) - np.where(fin, row_lse, 0.0)
+            p = np.zeros((Nq, Nk))
+            p[live] = np.exp(shifted[live])
+            dv[b, :, h, :] = p.T @ dom
+            dp = dom @ vm.T
+            rowdot = np.sum(dom * out[b, :, h, :], axis=1, keepdims=True)
+            ds = p * (dp - rowdot)
+            dq[b, :, h, :] = sc * (ds @ km)
+            dk[b, :, h, :] = sc * (ds.T @ qm)
     return dq, dk, dv
 
 

@@ -150,6 +150,22 @@ def test_merge_partials_argument_errors(lib):
     assert call(N=0) == FA_OK
 
 
+def test_accumulate_argument_errors(lib):
+    def call(acc=P16, part=P16, out=NULL, n=64):
+        return lib.fa_accumulate(acc, part, out, n, NULL)
+    assert call(n=-8) == INVALID
+    assert call(acc=NULL) == INVALID
+    assert call(part=NULL, out=NULL) == INVALID
+    assert b"both NULL" in lib.fa_last_error()
+    assert call(n=60) == INVALID
+    assert b"multiple of 8" in lib.fa_last_error()
+    assert call(part=P_ODD) == INVALID
+    assert call(out=P_ODD) == INVALID
+    assert call(acc=P_ODD, part=NULL, out=P16) == INVALID
+    # Nothing to add: a no-op, even with null pointers.
+    assert call(acc=NULL, part=NULL, n=0) == FA_OK
+
+
 def _dec(lib, q=P16, kn=NULL, vn=NULL, seq=P16, Ncap=2048, d=64, B=2):
     return lib.fa_decode(q, P16, P16, seq, kn, vn, P16, NULL, B, 16, Ncap, d, 1, 0.125, NULL, 0, S0)
 

@@ -1,6 +1,7 @@
 """Ring attention pieces on one GPU: the LSE merge kernel against the oracle's merge,
-and the full ring schedule for 1, 2 and 4 shards emulated in one process (the shard
-exchange becomes indexing) against the oracle's attention over the whole sequence."""
+the fp32 sum kernel of the backward, and the full ring schedule (forward and backward)
+for 1, 2 and 4 shards emulated in one process (the shard exchange becomes indexing)
+against the oracle's attention and gradients over the whole sequence."""
 import numpy as np
 import pytest
 import torch
@@ -8,8 +9,8 @@ import torch
 import exact_attention_155_b200 as fa
 import oracle
 from exact_attention_155_b200.inputs import bf16_randn, to_f64
-from exact_attention_155_b200.ring import ring_attention_fwd_emulated
-from helpers import LSE_ATOL, OUT_ATOL, check_fwd, default_scale, make_inputs
+from exact_attention_155_b200.ring import ring_attention_bwd_emulated, ring_attention_fwd_emulated
+from helpers import LSE_ATOL, OUT_ATOL, check_fwd, check_grads, default_scale, make_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -58,3 +59,43 @@ def test_emulated_ring_matches_whole_sequence(world, causal, d):
     out, lse = ring_attention_fwd_emulated(q, k, v, world, causal=causal, scale=sc)
     torch.cuda.synchronize()
     check_fwd(out, lse, inp, causal, sc)
+
+
+def test_accumulate_kernel_is_exact():
+    """fa_accumulate: one fp32 addition of an exactly converted bf16 term, and a
+    round-to-nearest-even bf16 copy; both are fixed to the bit."""
+    g = torch.Generator().manual_seed(9990)
+    acc = torch.randn((3, 77, 5, 64), generator=g, dtype=torch.float32).cuda()
+    part = bf16_randn((3, 77, 5, 64), g).cuda()
+    ref = acc + part.float()
+    out = torch.empty_like(part)
+    fa.ops.accumulate(acc, part, out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(acc, ref)
+    assert torch.equal(out, ref.to(torch.bfloat16))
+    out2 = torch.zeros_like(part)
+    fa.ops.accumulate(acc, None, out=out2)  # copy only: the sum is unchanged
+    torch.cuda.synchronize()
+    assert torch.equal(acc, ref) and torch.equal(out2, out)
+    with pytest.raises(ValueError):
+        fa.ops.accumulate(acc)
+    odd = torch.zeros(12, dtype=torch.float32, device="cuda")
+    with pytest.raises(fa.FAError):
+        fa.ops.accumulate(odd, torch.zeros(12, dtype=torch.bfloat16, device="cuda"))
+
+
+@pytest.mark.parametrize("world", [1, 2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_emulated_ring_bwd_matches_whole_sequence(world, causal, d):
+    """Ring backward for 1, 2 and 4 shards (the exchange emulated in one process): the
+    recomputed backward of every visited shard pair with the whole rows' LSE and
+    output, summed in fp32, against the oracle's gradients of the whole sequence."""
+    B, N, H = 1, 1024, 2
+    inp = make_inputs(B, N, H, d, 9990 + world + d + int(causal))
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    sc = default_scale(d)
+    out, lse = ring_attention_fwd_emulated(q, k, v, world, causal=causal, scale=sc)
+    grads = ring_attention_bwd_emulated(q, k, v, out, do, lse, world, causal=causal, scale=sc)
+    torch.cuda.synchronize()
+    check_grads(grads, inp, causal, sc)

@@ -70,42 +70,113 @@ def test_ring_exchange_delivers_scheduled_shards(world):
         assert got[rank] == [src for _, src, _ in ring_schedule(rank, world, False)]
 
 
-def _ring_worker(rank, world, port, causal, q):
-    """Runs ring_attention_fwd on CPU tensors over gloo with the per-block compute
-    replaced by the float64 oracle (a test seam: the product path calls the CUDA
-    library), and returns this rank's rows."""
+def _oracle_attend_and_merge(qs, ks, vs, mode, scale, o_acc, lse_acc, out, stream=None):
+    """Stand-in for ring._attend_and_merge on CPU tensors: the float64 oracle's
+    attention and merge (a test seam; the product path calls the CUDA library)."""
     import numpy as np
 
     import oracle
     from exact_attention_155_b200 import ring
+    _SEAM_CALLS.append(("fwd", mode, out is not None))
+    if mode == ring.SKIP:
+        return
+    to64 = lambda t: t.double().numpy()
+    o, l = oracle.attention_forward(to64(qs), to64(ks), to64(vs), causal=(mode == ring.CAUSAL),
+                                    scale=scale)
+    acc_o = o_acc.double().numpy()
+    acc_l = lse_acc.double().numpy()
+    mo, ml = oracle.merge_partials(np.stack([acc_o, o]),
+                                   np.stack([acc_l.transpose(0, 2, 1), l.transpose(0, 2, 1)]))
+    o_acc.copy_(torch.from_numpy(mo))
+    lse_acc.copy_(torch.from_numpy(ml.transpose(0, 2, 1)))
+    if out is not None:
+        out.copy_(o_acc)
 
-    def attend_and_merge(qs, ks, vs, mode, scale, o_acc, lse_acc, out, stream=None):
-        if mode == ring.SKIP:
-            return
-        to64 = lambda t: t.double().numpy()
-        o, l = oracle.attention_forward(to64(qs), to64(ks), to64(vs), causal=(mode == ring.CAUSAL),
-                                        scale=scale)
-        acc_o = o_acc.double().numpy()
-        acc_l = lse_acc.double().numpy()
-        mo, ml = oracle.merge_partials(np.stack([acc_o, o]),
-                                       np.stack([acc_l.transpose(0, 2, 1), l.transpose(0, 2, 1)]))
-        o_acc.copy_(torch.from_numpy(mo))
-        lse_acc.copy_(torch.from_numpy(ml.transpose(0, 2, 1)))
 
-    ring._attend_and_merge = attend_and_merge
+def _oracle_grad_terms(qs, ks, vs, out, dout, lse, mode, scale, dq_acc, dk_acc, dv_acc, dq_out,
+                       bufs, stream=None):
+    """Stand-in for ring._grad_terms on CPU tensors: the oracle's terms of one shard
+    pair, added to the running sums."""
+    import oracle
+    from exact_attention_155_b200 import ring
+    _SEAM_CALLS.append(("bwd", mode, dq_out is not None))
+    if mode == ring.SKIP:
+        return
+    to64 = lambda t: t.double().numpy()
+    tq, tk, tv = oracle.attention_backward_from_stats(
+        to64(qs), to64(ks), to64(vs), to64(out), to64(dout), to64(lse),
+        causal=(mode == ring.CAUSAL), scale=scale)
+    dq_acc += torch.from_numpy(tq).to(dq_acc.dtype)
+    dk_acc += torch.from_numpy(tk).to(dk_acc.dtype)
+    dv_acc += torch.from_numpy(tv).to(dv_acc.dtype)
+    if dq_out is not None:
+        dq_out.copy_(dq_acc)
+
+
+def _oracle_to_bf16(acc, out, stream=None):
+    _SEAM_CALLS.append(("convert", None, True))
+    out.copy_(acc)
+
+
+_SEAM_CALLS = []
+# The driver keeps its running sums in fp32 (as on the GPU); the seams compute in fp64.
+_ATOL = 1e-5
+
+
+def _use_oracle_seams(ring):
+    ring._attend_and_merge = _oracle_attend_and_merge
+    ring._grad_terms = _oracle_grad_terms
+    ring._to_bf16 = _oracle_to_bf16
+
+
+def _full_inputs(world, S=6, B=1, H=2, d=4, seed=123):
+    g = torch.Generator().manual_seed(seed)
+    return [torch.randn((B, S * world, H, d), generator=g, dtype=torch.float64) for _ in range(4)]
+
+
+def _ring_worker(rank, world, port, causal, q):
+    """Runs ring_attention_fwd on CPU tensors over gloo with the per-block compute
+    replaced by the float64 oracle, and returns this rank's rows."""
+    from exact_attention_155_b200 import ring
+
+    _use_oracle_seams(ring)
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world,
                             timeout=__import__("datetime").timedelta(seconds=60))
     try:
-        g = torch.Generator().manual_seed(123)
-        B, S, H, d = 1, 6, 2, 4
-        full = [torch.randn((B, S * world, H, d), generator=g) for _ in range(3)]
-        qs, ks, vs = (t[:, rank * S:(rank + 1) * S].contiguous() for t in full)
+        full = _full_inputs(world)
+        S = full[0].shape[1] // world
+        qs, ks, vs = (t[:, rank * S:(rank + 1) * S].contiguous() for t in full[:3])
         out, lse = ring.ring_attention_fwd(qs, ks, vs, causal=causal, scale=0.5)
-        q.put((rank, out.float().numpy(), lse.numpy(), [t.numpy() for t in full]))
+        q.put((rank, out.numpy(), lse.numpy(), [t.numpy() for t in full], list(_SEAM_CALLS)))
     finally:
         dist.destroy_process_group()
+
+
+def _check_out_written_once(calls, kind):
+    # The bf16 result is written by the last merge (or sum) that is not skipped, once.
+    writes = [i for i, c in enumerate(calls) if c[0] == kind and c[2]]
+    assert len(writes) == 1
+    later = [c for c in calls[writes[0] + 1:] if c[0] == kind]
+    assert all(c[1] == "skip" for c in later)
+
+
+def _spawn(target, world, *args):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=target, args=(r, world, port, *args, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = {}
+    for _ in range(world):
+        item = q.get(timeout=240)
+        got[item[0]] = item[1:]
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    return got
 
 
 @pytest.mark.parametrize("world", [2, 3])
@@ -114,24 +185,84 @@ def test_ring_attention_driver_over_gloo(world, causal):
     import numpy as np
 
     import oracle
-    ctx = mp.get_context("spawn")
-    q = ctx.Queue()
-    port = _free_port()
-    procs = [ctx.Process(target=_ring_worker, args=(r, world, port, causal, q)) for r in range(world)]
-    for p in procs:
-        p.start()
-    for p in procs:
-        p.join(180)
-        assert p.exitcode == 0
-    got = {}
-    for _ in range(world):
-        rank, o, l, full = q.get(timeout=10)
-        got[rank] = (o, l)
-    ref_o, ref_l = oracle.attention_forward(*[f.astype(np.float64) for f in full], causal=causal,
-                                            scale=0.5)
+    got = _spawn(_ring_worker, world, causal)
+    full = got[0][2]
+    ref_o, ref_l = oracle.attention_forward(*full[:3], causal=causal, scale=0.5)
     S = ref_o.shape[1] // world
     for rank in range(world):
-        o, l = got[rank]
-        # The driver's output is bf16; the LSE stays fp32 from the merges.
-        np.testing.assert_allclose(o, ref_o[:, rank * S:(rank + 1) * S], atol=2e-2)
-        np.testing.assert_allclose(l, ref_l[:, :, rank * S:(rank + 1) * S], atol=1e-6)
+        o, l, _, calls = got[rank]
+        _check_out_written_once(calls, "fwd")
+        np.testing.assert_allclose(o, ref_o[:, rank * S:(rank + 1) * S], atol=_ATOL)
+        np.testing.assert_allclose(l, ref_l[:, :, rank * S:(rank + 1) * S], atol=_ATOL)
+
+
+def _ring_bwd_worker(rank, world, port, causal, q):
+    """Runs ring_attention_bwd on CPU tensors over gloo with the per-pair compute
+    replaced by the oracle, from the oracle's whole-sequence forward (what the ring
+    forward returns); returns this rank's gradients."""
+    import oracle
+    from exact_attention_155_b200 import ring
+
+    _use_oracle_seams(ring)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        full = _full_inputs(world, seed=321)
+        out, lse = oracle.attention_forward(*[t.numpy() for t in full[:3]], causal=causal,
+                                            scale=0.5)
+        S = out.shape[1] // world
+        rows = lambda t: t[:, rank * S:(rank + 1) * S].contiguous()
+        qs, ks, vs, dos = (rows(t) for t in full)
+        os_ = rows(torch.from_numpy(out))
+        ls = torch.from_numpy(lse[:, :, rank * S:(rank + 1) * S]).contiguous()
+        dq, dk, dv = ring.ring_attention_bwd(qs, ks, vs, os_, dos, ls, causal=causal, scale=0.5)
+        q.put((rank, [g.numpy() for g in (dq, dk, dv)], [t.numpy() for t in full],
+               list(_SEAM_CALLS)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_attention_bwd_driver_over_gloo(world, causal):
+    """dQ stays home, the dK/dV sums travel a full turn: each rank ends with the
+    whole-sequence gradients of its own shards."""
+    import numpy as np
+
+    import oracle
+    got = _spawn(_ring_bwd_worker, world, causal)
+    full = got[0][1]
+    refs = oracle.attention_backward(*full, causal=causal, scale=0.5)
+    S = refs[0].shape[1] // world
+    for rank in range(world):
+        grads, _, calls = got[rank]
+        _check_out_written_once(calls, "bwd")
+        assert [c for c in calls if c[0] == "convert"] == [("convert", None, True)] * 2
+        for g, r in zip(grads, refs):
+            np.testing.assert_allclose(g, r[:, rank * S:(rank + 1) * S], atol=_ATOL)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulated_ring_fwd_and_bwd_on_cpu(world, causal, monkeypatch):
+    """The one-process emulation's bookkeeping (shard slicing, the per-shard sums, the
+    step that writes each result) with the oracle standing in for the kernels."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_155_b200 import ring
+    monkeypatch.setattr(ring, "_attend_and_merge", _oracle_attend_and_merge)
+    monkeypatch.setattr(ring, "_grad_terms", _oracle_grad_terms)
+    monkeypatch.setattr(ring, "_to_bf16", _oracle_to_bf16)
+    full = _full_inputs(world, seed=99 + world)
+    q, k, v, do = full
+    out, lse = ring.ring_attention_fwd_emulated(q, k, v, world, causal=causal, scale=0.7)
+    ref_o, ref_l = oracle.attention_forward(*[t.numpy() for t in full[:3]], causal=causal, scale=0.7)
+    np.testing.assert_allclose(out.numpy(), ref_o, atol=_ATOL)
+    np.testing.assert_allclose(lse.numpy(), ref_l, atol=_ATOL)
+    grads = ring.ring_attention_bwd_emulated(q, k, v, out, do, lse, world, causal=causal, scale=0.7)
+    refs = oracle.attention_backward(*[t.numpy() for t in full], causal=causal, scale=0.7)
+    for g, r in zip(grads, refs):
+        np.testing.assert_allclose(g.numpy(), r, atol=_ATOL)
