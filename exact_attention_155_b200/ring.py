@@ -48,11 +48,14 @@ def ring_schedule(rank: int, world: int, causal: bool) -> List[Tuple[int, int, s
 
 
 def ring_pass(send: torch.Tensor, recv: torch.Tensor, rank: int, world: int, group=None):
-    """Start sending `send` to rank + 1 and receiving rank - 1's buffer into `recv`;
-    returns the requests to wait on."""
+    """Start sending `send` to rank + 1 and receiving rank - 1's buffer into `recv`
+    (ranks within `group`); returns the requests to wait on."""
     import torch.distributed as dist
-    ops_ = [dist.P2POp(dist.isend, send, (rank + 1) % world, group),
-            dist.P2POp(dist.irecv, recv, (rank - 1) % world, group)]
+
+    def peer(r):  # point-to-point calls take global ranks
+        return r if group is None else dist.get_global_rank(group, r)
+    ops_ = [dist.P2POp(dist.isend, send, peer((rank + 1) % world), group),
+            dist.P2POp(dist.irecv, recv, peer((rank - 1) % world), group)]
     return dist.batch_isend_irecv(ops_)
 
 

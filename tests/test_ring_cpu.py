@@ -163,6 +163,9 @@ def _check_out_written_once(calls, kind):
 
 
 def _spawn(target, world, *args):
+    """Runs target(rank, world, port, *args, queue) in `world` spawned processes and
+    returns {rank: rest of the tuple the rank put on the queue}. A rank that hangs or
+    dies fails the test within a few minutes; the children are always reaped."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
@@ -170,11 +173,17 @@ def _spawn(target, world, *args):
     for p in procs:
         p.start()
     got = {}
-    for _ in range(world):
-        item = q.get(timeout=240)
-        got[item[0]] = item[1:]
+    try:
+        for _ in range(world):
+            item = q.get(timeout=120)
+            got[item[0]] = item[1:]
+    finally:
+        for p in procs:
+            p.join(60 if len(got) == world else 1)
+            if p.is_alive():
+                p.terminate()
+                p.join(10)
     for p in procs:
-        p.join(120)
         assert p.exitcode == 0
     return got
 
@@ -266,3 +275,53 @@ def test_emulated_ring_fwd_and_bwd_on_cpu(world, causal, monkeypatch):
     refs = oracle.attention_backward(*[t.numpy() for t in full], causal=causal, scale=0.7)
     for g, r in zip(grads, refs):
         np.testing.assert_allclose(g.numpy(), r, atol=_ATOL)
+
+
+def _subgroup_worker(rank, world, port, q):
+    """Ranks 1 and 3 of four run the ring (forward, then backward) over a process
+    subgroup; ranks 0 and 2 only take part in creating it."""
+    from exact_attention_155_b200 import ring
+
+    _use_oracle_seams(ring)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        members = [1, 3]
+        grp = dist.new_group(members)
+        if rank in members:
+            gr = members.index(rank)
+            full = _full_inputs(2, seed=555)
+            S = full[0].shape[1] // 2
+            qs, ks, vs, dos = (t[:, gr * S:(gr + 1) * S].contiguous() for t in full)
+            out, lse = ring.ring_attention_fwd(qs, ks, vs, causal=True, scale=0.5, group=grp)
+            grads = ring.ring_attention_bwd(qs, ks, vs, out, dos, lse, causal=True, scale=0.5,
+                                            group=grp)
+            q.put((rank, gr, out.numpy(), lse.numpy(), [g.numpy() for g in grads],
+                   [t.numpy() for t in full]))
+        else:
+            q.put((rank, None, None, None, None, None))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_over_a_process_subgroup():
+    """Point-to-point peers are global ranks: a ring over ranks {1, 3} must exchange
+    between 1 and 3, not between group ranks 0 and 1."""
+    import numpy as np
+
+    import oracle
+    got = _spawn(_subgroup_worker, 4)
+    full = got[1][4]
+    ref_o, ref_l = oracle.attention_forward(*full[:3], causal=True, scale=0.5)
+    refs = oracle.attention_backward(*full, causal=True, scale=0.5)
+    S = ref_o.shape[1] // 2
+    for rank in (1, 3):
+        gr, o, l, grads, _ = got[rank]
+        rows = slice(gr * S, (gr + 1) * S)
+        np.testing.assert_allclose(o, ref_o[:, rows], atol=_ATOL)
+        np.testing.assert_allclose(l, ref_l[:, :, rows], atol=_ATOL)
+        for g, r in zip(grads, refs):
+            np.testing.assert_allclose(g, r[:, rows], atol=_ATOL)
