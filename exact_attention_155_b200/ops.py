@@ -120,15 +120,41 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _require(t: torch.Tensor, name: str, dtype=torch.bfloat16):
+def _device_ctx(device):
+    """Makes `device` current for the call (the library launches on the current device)."""
+    return torch.cuda.device(device)
+
+
+# Device type every tensor handed to the library must have.
+_DEVICE_TYPE = "cuda"
+
+
+def _require(t: torch.Tensor, name: str, dtype=torch.bfloat16, shape=None, device=None):
+    """Checks a tensor the library will read or write: a contiguous tensor of `dtype` on
+    the library's device type, and, when given, exactly `shape` and on `device` (the
+    kernels index every buffer from the sizes alone, so a wrong shape or another GPU's
+    buffer must never reach them)."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
+    if t.device.type != _DEVICE_TYPE:
         raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype} (got {t.dtype}); inputs and outputs share one dtype")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device} like the other operands (got {t.device})")
+
+
+def _workspace(workspace, need: int, device):
+    """The caller's workspace (uint8, contiguous, on `device`; the library checks its
+    size) or a new one of `need` bytes."""
+    if workspace is None:
+        return torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    _require(workspace, "workspace", torch.uint8, device=device)
+    return workspace
 
 
 def _scale(scale, d):
@@ -142,20 +168,21 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
 
     Returns (out [B, N, H, d] bf16, lse [B, H, N] fp32). scale=None -> 1/sqrt(d).
     """
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        _require(t, name)
-    if q.dim() != 4 or k.shape != q.shape or v.shape != q.shape:
-        raise ValueError(f"q, k, v must all be [B, N, H, d] with equal shapes "
-                         f"(got {tuple(q.shape)}, {tuple(k.shape)}, {tuple(v.shape)})")
+    _require(q, "q")
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, N, H, d] (got {tuple(q.shape)})")
+    dev = q.device
+    for name, t in (("k", k), ("v", v)):
+        _require(t, name, shape=q.shape, device=dev)
     B, N, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     if lse is None:
-        lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    _require(out, "out")
-    _require(lse, "lse", torch.float32)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    _require(out, "out", shape=q.shape, device=dev)
+    _require(lse, "lse", torch.float32, shape=(B, H, N), device=dev)
     lib = load_library()
-    with torch.cuda.device(q.device):
+    with _device_ctx(dev):
         _check(lib.fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, H, N, d,
                           int(bool(causal)), _scale(scale, d), _stream(stream)))
     return out, lse
@@ -172,24 +199,22 @@ def bwd(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = 
     main_events: optional (start, stop) torch.cuda.Event pair recorded around the main
     backward kernel (fa_bwd_profiled), for timing that kernel on its own stream.
     """
-    for name, t in (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout)):
-        _require(t, name)
-        if t.shape != q.shape:
-            raise ValueError(f"{name} must have q's shape {tuple(q.shape)}")
-    _require(lse, "lse", torch.float32)
+    _require(q, "q")
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, N, H, d] (got {tuple(q.shape)})")
+    dev = q.device
+    for name, t in (("k", k), ("v", v), ("out", out), ("dout", dout)):
+        _require(t, name, shape=q.shape, device=dev)
     B, N, H, d = q.shape
-    if tuple(lse.shape) != (B, H, N):
-        raise ValueError(f"lse must be [B, H, N] = {(B, H, N)}")
+    _require(lse, "lse", torch.float32, shape=(B, H, N), device=dev)
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
     for name, t in (("dq", dq), ("dk", dk), ("dv", dv)):
-        _require(t, name)
+        _require(t, name, shape=q.shape, device=dev)
     lib = load_library()
-    need = int(lib.fa_bwd_workspace_size(B, H, N, d))
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    with torch.cuda.device(q.device):
+    workspace = _workspace(workspace, int(lib.fa_bwd_workspace_size(B, H, N, d)), dev)
+    with _device_ctx(dev):
         if main_events is None:
             _check(lib.fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
                               _ptr(dq), _ptr(dk), _ptr(dv), B, H, N, d, int(bool(causal)),
@@ -208,13 +233,15 @@ def bwd(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = 
     return dq, dk, dv
 
 
-def _row_stride(t: torch.Tensor, name: str, varlen: bool, shape) -> int:
+def _row_stride(t: torch.Tensor, name: str, varlen: bool, shape, device=None) -> int:
     """Elements between consecutive tokens of a [B, N, H, d] (or [total, H, d]) view
     whose (H, d) block is contiguous; raises for any other layout."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != "cuda":
+    if t.device.type != _DEVICE_TYPE:
         raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device} like the other operands (got {t.device})")
     if t.dtype != torch.bfloat16:
         raise ValueError(f"{name} must be torch.bfloat16 (got {t.dtype}); inputs and outputs share one dtype")
     if tuple(t.shape) != tuple(shape):
@@ -234,6 +261,26 @@ def _window(window):
     return wl, wr
 
 
+def _ex_layout(q, cu_seqlens, max_seqlen):
+    """(varlen, B, N, H, d, total, shape) of an extended call from q and cu_seqlens."""
+    varlen = cu_seqlens is not None
+    if varlen:
+        _require(cu_seqlens, "cu_seqlens", torch.int32, device=q.device)
+        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
+            raise ValueError("cu_seqlens must be int32 [B + 1]")
+        if max_seqlen is None:
+            raise ValueError("max_seqlen is required with cu_seqlens")
+        if q.dim() != 3:
+            raise ValueError(f"q must be [total, H, d] with cu_seqlens (got {tuple(q.shape)})")
+        total, H, d = q.shape
+        B, N = cu_seqlens.numel() - 1, int(max_seqlen)
+        return True, B, N, H, d, total, (total, H, d)
+    if q.dim() != 4:
+        raise ValueError(f"q must be [B, N, H, d] (got {tuple(q.shape)})")
+    B, N, H, d = q.shape
+    return False, B, N, H, d, 0, (B, N, H, d)
+
+
 def fwd_ex(q, k, v, causal: bool = False, scale: Optional[float] = None, window=None,
            cu_seqlens: Optional[torch.Tensor] = None, max_seqlen: Optional[int] = None,
            out=None, lse=None, stream=None):
@@ -246,33 +293,21 @@ def fwd_ex(q, k, v, causal: bool = False, scale: Optional[float] = None, window=
     window = (left, right): query i sees keys [i - left, i + right], -1 = unbounded;
     causal fixes right = 0. Returns (out, lse); out is contiguous unless given.
     """
-    varlen = cu_seqlens is not None
-    if varlen:
-        _require(cu_seqlens, "cu_seqlens", torch.int32)
-        if cu_seqlens.dim() != 1 or cu_seqlens.numel() < 1:
-            raise ValueError("cu_seqlens must be int32 [B + 1]")
-        if max_seqlen is None:
-            raise ValueError("max_seqlen is required with cu_seqlens")
-        total, H, d = q.shape
-        B, N = cu_seqlens.numel() - 1, int(max_seqlen)
-        shape = (total, H, d)
-    else:
-        B, N, H, d = q.shape
-        total = 0
-        shape = (B, N, H, d)
-    rs = [_row_stride(t, n, varlen, shape) for n, t in (("q", q), ("k", k), ("v", v))]
+    if not isinstance(q, torch.Tensor):
+        raise TypeError("q must be a torch.Tensor")
+    dev = q.device
+    varlen, B, N, H, d, total, shape = _ex_layout(q, cu_seqlens, max_seqlen)
+    rs = [_row_stride(t, n, varlen, shape, dev) for n, t in (("q", q), ("k", k), ("v", v))]
     if out is None:
-        out = torch.empty(shape, dtype=torch.bfloat16, device=q.device)
-    rs.append(_row_stride(out, "out", varlen, shape))
+        out = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+    rs.append(_row_stride(out, "out", varlen, shape, dev))
     lse_shape = (H, total) if varlen else (B, H, N)
     if lse is None:
-        lse = torch.empty(lse_shape, dtype=torch.float32, device=q.device)
-    _require(lse, "lse", torch.float32)
-    if tuple(lse.shape) != lse_shape:
-        raise ValueError(f"lse must be {lse_shape}")
+        lse = torch.empty(lse_shape, dtype=torch.float32, device=dev)
+    _require(lse, "lse", torch.float32, shape=lse_shape, device=dev)
     wl, wr = _window(window)
     lib = load_library()
-    with torch.cuda.device(q.device):
+    with _device_ctx(dev):
         _check(lib.fa_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), _ptr(cu_seqlens),
                              total, B, H, N, d, rs[0], rs[1], rs[2], rs[3], int(bool(causal)),
                              wl, wr, _scale(scale, d), _stream(stream)))
@@ -284,34 +319,22 @@ def bwd_ex(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float]
            max_seqlen: Optional[int] = None, dq=None, dk=None, dv=None, workspace=None,
            stream=None):
     """Backward of fwd_ex (fa_bwd_ex): same layouts and options. Returns (dq, dk, dv)."""
-    varlen = cu_seqlens is not None
-    if varlen:
-        _require(cu_seqlens, "cu_seqlens", torch.int32)
-        if max_seqlen is None:
-            raise ValueError("max_seqlen is required with cu_seqlens")
-        total, H, d = q.shape
-        B, N = cu_seqlens.numel() - 1, int(max_seqlen)
-        shape = (total, H, d)
-    else:
-        B, N, H, d = q.shape
-        total = 0
-        shape = (B, N, H, d)
-    dq = torch.empty(shape, dtype=torch.bfloat16, device=q.device) if dq is None else dq
-    dk = torch.empty(shape, dtype=torch.bfloat16, device=q.device) if dk is None else dk
-    dv = torch.empty(shape, dtype=torch.bfloat16, device=q.device) if dv is None else dv
+    if not isinstance(q, torch.Tensor):
+        raise TypeError("q must be a torch.Tensor")
+    dev = q.device
+    varlen, B, N, H, d, total, shape = _ex_layout(q, cu_seqlens, max_seqlen)
+    dq = torch.empty(shape, dtype=torch.bfloat16, device=dev) if dq is None else dq
+    dk = torch.empty(shape, dtype=torch.bfloat16, device=dev) if dk is None else dk
+    dv = torch.empty(shape, dtype=torch.bfloat16, device=dev) if dv is None else dv
     names = (("q", q), ("k", k), ("v", v), ("out", out), ("dout", dout), ("dq", dq), ("dk", dk),
              ("dv", dv))
-    rs = (_c_ll * 8)(*[_row_stride(t, n, varlen, shape) for n, t in names])
-    _require(lse, "lse", torch.float32)
+    rs = (_c_ll * 8)(*[_row_stride(t, n, varlen, shape, dev) for n, t in names])
     lse_shape = (H, total) if varlen else (B, H, N)
-    if tuple(lse.shape) != lse_shape:
-        raise ValueError(f"lse must be {lse_shape}")
+    _require(lse, "lse", torch.float32, shape=lse_shape, device=dev)
     wl, wr = _window(window)
     lib = load_library()
-    need = int(lib.fa_bwd_workspace_size(B, H, N, d))
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
-    with torch.cuda.device(q.device):
+    workspace = _workspace(workspace, int(lib.fa_bwd_workspace_size(B, H, N, d)), dev)
+    with _device_ctx(dev):
         _check(lib.fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens), total, B, H, N, d, rs,
                              int(bool(causal)), wl, wr, _scale(scale, d), _ptr(workspace),
@@ -323,9 +346,9 @@ def fwd_qkvpacked(qkv, causal: bool = False, scale: Optional[float] = None, wind
                   stream=None):
     """Forward on a packed [B, N, 3, H, d] tensor (flash_attn_qkvpacked_func layout),
     read in place through row strides. Returns (out [B, N, H, d], lse [B, H, N])."""
+    _require(qkv, "qkv")
     if qkv.dim() != 5 or qkv.shape[2] != 3:
         raise ValueError("qkv must be [B, N, 3, H, d]")
-    _require(qkv, "qkv")
     return fwd_ex(qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], causal=causal, scale=scale,
                   window=window, stream=stream)
 
@@ -333,11 +356,11 @@ def fwd_qkvpacked(qkv, causal: bool = False, scale: Optional[float] = None, wind
 def bwd_qkvpacked(qkv, out, dout, lse, causal: bool = False, scale: Optional[float] = None,
                   window=None, dqkv=None, stream=None):
     """Backward of fwd_qkvpacked; the gradient is written packed, [B, N, 3, H, d]."""
+    _require(qkv, "qkv")
     if qkv.dim() != 5 or qkv.shape[2] != 3:
         raise ValueError("qkv must be [B, N, 3, H, d]")
-    _require(qkv, "qkv")
     dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
-    _require(dqkv, "dqkv")
+    _require(dqkv, "dqkv", shape=qkv.shape, device=qkv.device)
     bwd_ex(qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], out, dout, lse, causal=causal, scale=scale,
            window=window, dq=dqkv[:, :, 0], dk=dqkv[:, :, 1], dv=dqkv[:, :, 2], stream=stream)
     return dqkv
@@ -345,6 +368,26 @@ def bwd_qkvpacked(qkv, out, dout, lse, causal: bool = False, scale: Optional[flo
 
 def decode_workspace_size(B: int, H: int, Ncap: int, d: int) -> int:
     return int(load_library().fa_decode_workspace_size(B, H, Ncap, d))
+
+
+def _decode_step_args(q, cache_seqlens, k_new, v_new, out, lse):
+    """Checks shared by the decode calls; returns (B, H, d, out, lse)."""
+    _require(q, "q")
+    if q.dim() != 4 or q.shape[1] != 1:
+        raise ValueError(f"q must be [B, 1, H, d] (got {tuple(q.shape)})")
+    dev = q.device
+    B, _, H, d = q.shape
+    _require(cache_seqlens, "cache_seqlens", torch.int32, shape=(B,), device=dev)
+    if (k_new is None) != (v_new is None):
+        raise ValueError("k_new and v_new must be given together")
+    if k_new is not None:
+        _require(k_new, "k_new", shape=q.shape, device=dev)
+        _require(v_new, "v_new", shape=q.shape, device=dev)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H), dtype=torch.float32, device=dev) if lse is None else lse
+    _require(out, "out", shape=q.shape, device=dev)
+    _require(lse, "lse", torch.float32, shape=(B, H), device=dev)
+    return B, H, d, out, lse
 
 
 def decode(q, k_cache, v_cache, cache_seqlens, k_new=None, v_new=None, causal: bool = True,
@@ -355,34 +398,19 @@ def decode(q, k_cache, v_cache, cache_seqlens, k_new=None, v_new=None, causal: b
     device (valid rows before the append). With k_new / v_new ([B, 1, H, d]) the row is
     appended at cache_seqlens[b]. Returns (out [B, 1, H, d] bf16, lse [B, H] fp32).
     """
-    _require(q, "q")
-    _require(k_cache, "k_cache")
-    _require(v_cache, "v_cache")
-    _require(cache_seqlens, "cache_seqlens", torch.int32)
-    B, one, H, d = q.shape
-    if one != 1 or k_cache.dim() != 4 or k_cache.shape != v_cache.shape \
-            or k_cache.shape[0] != B or k_cache.shape[2] != H or k_cache.shape[3] != d:
+    B, H, d, out, lse = _decode_step_args(q, cache_seqlens, k_new, v_new, out, lse)
+    dev = q.device
+    _require(k_cache, "k_cache", device=dev)
+    if k_cache.dim() != 4 or k_cache.shape[0] != B or k_cache.shape[2] != H or k_cache.shape[3] != d:
         raise ValueError("q must be [B,1,H,d] and caches [B,Ncap,H,d]")
-    if tuple(cache_seqlens.shape) != (B,):
-        raise ValueError("cache_seqlens must be int32 [B]")
+    _require(v_cache, "v_cache", shape=k_cache.shape, device=dev)
     Ncap = k_cache.shape[1]
-    if (k_new is None) != (v_new is None):
-        raise ValueError("k_new and v_new must be given together")
-    if k_new is not None:
-        _require(k_new, "k_new")
-        _require(v_new, "v_new")
-        if k_new.shape != q.shape or v_new.shape != q.shape:
-            raise ValueError("k_new and v_new must be [B, 1, H, d]")
-    out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
-    _require(out, "out")
-    _require(lse, "lse", torch.float32)
     lib = load_library()
     need = int(lib.fa_decode_workspace_size(B, H, Ncap, d))
-    if workspace is None and need > 0:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace is not None or need > 0:
+        workspace = _workspace(workspace, need, dev)
     ws_bytes = 0 if workspace is None else workspace.numel()
-    with torch.cuda.device(q.device):
+    with _device_ctx(dev):
         _check(lib.fa_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(cache_seqlens),
                              _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(lse), B, H, Ncap, d,
                              int(bool(causal)), _scale(scale, d), _ptr(workspace), ws_bytes,
@@ -398,31 +426,18 @@ def decode_paged(q, k_pages, v_pages, block_table, cache_seqlens, k_new=None, v_
     q: [B, 1, H, d]; k_pages, v_pages: [num_pages, page_size, H, d]; block_table: int32
     [B, max_blocks] on the device; cache_seqlens: int32 [B] on the device. Returns
     (out [B, 1, H, d] bf16, lse [B, H] fp32)."""
-    _require(q, "q")
-    _require(k_pages, "k_pages")
-    _require(v_pages, "v_pages")
-    _require(block_table, "block_table", torch.int32)
-    _require(cache_seqlens, "cache_seqlens", torch.int32)
-    B, one, H, d = q.shape
-    if one != 1 or k_pages.dim() != 4 or k_pages.shape != v_pages.shape \
-            or k_pages.shape[2] != H or k_pages.shape[3] != d:
+    B, H, d, out, lse = _decode_step_args(q, cache_seqlens, k_new, v_new, out, lse)
+    dev = q.device
+    _require(k_pages, "k_pages", device=dev)
+    if k_pages.dim() != 4 or k_pages.shape[2] != H or k_pages.shape[3] != d:
         raise ValueError("q must be [B,1,H,d] and pages [num_pages,page_size,H,d]")
+    _require(v_pages, "v_pages", shape=k_pages.shape, device=dev)
+    _require(block_table, "block_table", torch.int32, device=dev)
     if block_table.dim() != 2 or block_table.shape[0] != B:
         raise ValueError("block_table must be int32 [B, max_blocks]")
-    if tuple(cache_seqlens.shape) != (B,):
-        raise ValueError("cache_seqlens must be int32 [B]")
     num_pages, page_size = k_pages.shape[0], k_pages.shape[1]
-    if (k_new is None) != (v_new is None):
-        raise ValueError("k_new and v_new must be given together")
-    if k_new is not None:
-        _require(k_new, "k_new")
-        _require(v_new, "v_new")
-    out = torch.empty_like(q) if out is None else out
-    lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if lse is None else lse
-    _require(out, "out")
-    _require(lse, "lse", torch.float32)
     lib = load_library()
-    with torch.cuda.device(q.device):
+    with _device_ctx(dev):
         _check(lib.fa_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
                                    block_table.shape[1], page_size, num_pages, _ptr(cache_seqlens),
                                    _ptr(k_new), _ptr(v_new), _ptr(out), _ptr(lse), B, H, d,
@@ -434,18 +449,18 @@ def merge_partials(o_acc, lse_acc, o_part, lse_part, out=None, stream=None):
     """Fold a partial result (o_part bf16 [B, N, H, d], lse_part [B, H, N]) into the
     running one (o_acc fp32 [B, N, H, d], lse_acc [B, H, N]) in place (fa_merge_partials);
     optionally write the merged output as bf16 into `out`."""
-    _require(o_acc, "o_acc", torch.float32)
-    _require(lse_acc, "lse_acc", torch.float32)
     _require(o_part, "o_part")
-    _require(lse_part, "lse_part", torch.float32)
+    if o_part.dim() != 4:
+        raise ValueError("o_part must be [B, N, H, d]")
+    dev = o_part.device
     B, N, H, d = o_part.shape
-    if o_acc.shape != o_part.shape or tuple(lse_acc.shape) != (B, H, N) \
-            or tuple(lse_part.shape) != (B, H, N):
-        raise ValueError("o_acc/o_part must be [B, N, H, d] and lse_acc/lse_part [B, H, N]")
+    _require(o_acc, "o_acc", torch.float32, shape=o_part.shape, device=dev)
+    _require(lse_acc, "lse_acc", torch.float32, shape=(B, H, N), device=dev)
+    _require(lse_part, "lse_part", torch.float32, shape=(B, H, N), device=dev)
     if out is not None:
-        _require(out, "out")
+        _require(out, "out", shape=o_part.shape, device=dev)
     lib = load_library()
-    with torch.cuda.device(o_acc.device):
+    with _device_ctx(dev):
         _check(lib.fa_merge_partials(_ptr(o_acc), _ptr(lse_acc), _ptr(o_part), _ptr(lse_part),
                                      _ptr(out), B, N, H, d, _stream(stream)))
     return o_acc, lse_acc
@@ -459,11 +474,9 @@ def accumulate(acc, part=None, out=None, stream=None):
         raise ValueError("give part, out or both")
     for name, t in (("part", part), ("out", out)):
         if t is not None:
-            _require(t, name)
-            if t.shape != acc.shape or t.device != acc.device:
-                raise ValueError(f"{name} must have acc's shape and device")
+            _require(t, name, shape=acc.shape, device=acc.device)
     lib = load_library()
-    with torch.cuda.device(acc.device):
+    with _device_ctx(acc.device):
         _check(lib.fa_accumulate(_ptr(acc), _ptr(part), _ptr(out), acc.numel(), _stream(stream)))
     return acc
 
