@@ -194,7 +194,10 @@ struct BwdLayout {
   static constexpr int kDQFree = kSFull + 6;
   static constexpr int kMmaDone = kSFull + 7;
   static constexpr int kDrain = kSFull + 8;
-  static constexpr int kNumBars = kDrain + 1;
+  // [4] per TMEM lane quarter: the first warpgroup's warp of the quarter has loaded
+  // S^T (the second warpgroup's P^T overwrites S^T columns that warp reads).
+  static constexpr int kSLoaded = kDrain + 1;
+  static constexpr int kNumBars = kSLoaded + 4;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kThreads = 448;
@@ -307,6 +310,7 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(BAR(L::kDQFree), 128);
     mbar_init(BAR(L::kMmaDone), 1);
     mbar_init(BAR(L::kDrain), 1);
+    for (int q = 0; q < 4; ++q) mbar_init(BAR(L::kSLoaded + q), 32);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -493,6 +497,10 @@ __global__ void __launch_bounds__(448, 1)
       tmem_wait_ld();
       reg_fence32(s0);
       reg_fence32(s1);
+      if (half == 0) {
+        tc_fence_before();
+        mbar_arrive(BAR(L::kSLoaded + wq));
+      }
       FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 1));
       // Local columns c in [qlo_c, qhi_c] are the queries that see this key (window
       // [key - wr, key + wl]); none if the key is past the sequence. Queries past the
@@ -517,6 +525,16 @@ __global__ void __launch_bounds__(448, 1)
         const float p1 = (c + 1 < qlo_c || c + 1 > qhi_c) ? 0.f : e1;
         pk[c2] = pack_bf16x2(p0, p1);
       }
+      // P^T of queries [c0, c0 + 64) goes to columns [c0/2, c0/2 + 32): for the second
+      // warpgroup those are S^T columns of the first one, which must have loaded them.
+      // (The first warpgroup overwrites only its own columns; it is never more than one
+      // tile ahead, since S^T(n + 1) waits for both warpgroups' P^T(n).)
+      if (half == 1) {
+        if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kSLoaded + wq), n & 1, abort_flag,
+                                                    kSiteBwdSoftmax))))
+          break;
+      }
+      tc_fence_after();
       tmem_st32(tS + lane_off + c0 / 2, pk);  // P^T bf16: two queries per 32-bit column
       tmem_wait_st();
       tc_fence_before();

@@ -443,6 +443,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int c = 0; c < 32; ++c) x[32 * q32 + c] = __uint_as_float(s0[c]);
           }
         }
+        tc_fence_before();  // the loads above precede the barrier that lets P be stored
         FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 1));
         const int kbase = j * 128 + C * grp;  // key index of this group's column 0
         // A tile needs per-element masking if it reaches past the sequence or outside
@@ -460,14 +461,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         // x holds raw scores (unmasked tile) or scaled, masked scores (masked tile).
         // exps(ms): p = 2^(x*sl2 - ms) (resp. 2^(x - ms)) for this group's C columns,
-        // their sum into rsum, and bf16 P into TMEM.
+        // their sum into rsum, and bf16 P (two keys per 32-bit word) into pk. store_p()
+        // writes pk to TMEM. P of keys [k, k + 32) lands in the S columns of keys
+        // [k/2, k/2 + 16), which another column group of the same rows may not have
+        // loaded yet, so P is stored only after a barrier over the row's groups: the
+        // vote (fast path) or the max exchange (exact path), both after every load.
         float rsum = 0.f;
+        uint32_t pk[C / 32][16];
         auto exps = [&](float ms) {
           const float nms = -ms;
           float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int ch = 0; ch < C / 32; ++ch) {
-            uint32_t pk[16];
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const int c = ch * 32 + 2 * i;
@@ -485,11 +490,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 bb = ex2_approx(bb);
               }
               add2(rs[2 * (i & 1)], rs[2 * (i & 1) + 1], rs[2 * (i & 1)], rs[2 * (i & 1) + 1], a, bb);
-              pk[i] = kAluPack ? pack_bf16x2_alu(a, bb) : pack_bf16x2(a, bb);
+              pk[ch][i] = kAluPack ? pack_bf16x2_alu(a, bb) : pack_bf16x2(a, bb);
             }
-            tmem_st16(tS + (C / 2) * grp + ch * 16, pk);  // P: two keys per 32-bit column
           }
           rsum = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        };
+        auto store_p = [&]() {
+          tc_fence_after();
+#pragma unroll
+          for (int ch = 0; ch < C / 32; ++ch) tmem_st16(tS + (C / 2) * grp + ch * 16, pk[ch]);
         };
         // Fast path: exponentiate against the current reference max. If this group's
         // exponentials of every row sum to at most 256, none of them exceeds 2^8, so P
@@ -506,7 +515,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!exact) {
           exps(m[t]);
           exact = named_bar_or(kBarVote, NTQ, !w_ok || !(rsum <= 256.f));
-          if (!exact) l[t] += rsum;
+          if (!exact) {
+            l[t] += rsum;
+            store_p();
+          }
         }
         if (exact) {
           // Exact path (first tile, negative scale, a grown row, or an abort): the
@@ -568,6 +580,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           named_bar_sync(kBarVote, NTQ);
           exps(m[t] == -INFINITY ? 0.f : m[t]);
           l[t] += rsum;
+          store_p();
         }
         FA_TRACE_EVENT(tr, FA_FWD_TR(1 + 4 * t + wq, j, 2));
         tmem_wait_st();
