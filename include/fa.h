@@ -158,7 +158,7 @@ fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out
  * no access to the application's allocator, or a latency-critical loop that must
  * not call an allocator (which may synchronise the device). This entry point takes
  * the same inputs and outputs as fa_bwd, minus the workspace, and uses a scratch
- * array that lives inside the library instead. The paper has no counterpart to
+ * array that lives inside the library instead. The FlashAttention pages have no counterpart to
  * this call; it only exists for such callers.
  *
  * Limits and behaviour:
