@@ -340,7 +340,7 @@ def run_ours(args, rank, world, local_rank):
         "peak_gbs": L2_REDUCTION_GBS,
         "frac": red_bytes / (bwd_main_ms * 1e-3) / 1e9 / L2_REDUCTION_GBS,
         "peak_kind": "bulk fp32 reduction rate measured by csrc/l2_reduction_rate.cu (all SMs, "
-                     "16.8 B/clk/SM into a 256 MiB buffer); not in the driver's peak file"}
+                     "16.8 B/clk/SM into a 256 MiB buffer); not one of the peaks in MEASURED_PEAKS.json"}
 
     # ---- end to end through the public API from pinned host buffers
     # Every step copies its own inputs host->device and its results device->host.
