@@ -325,3 +325,89 @@ def test_ring_over_a_process_subgroup():
         np.testing.assert_allclose(l, ref_l[:, :, rows], atol=_ATOL)
         for g, r in zip(grads, refs):
             np.testing.assert_allclose(g, r[:, rows], atol=_ATOL)
+
+
+class _AbiStandIns:
+    """CPU stand-ins for the binding calls the ring driver makes (fwd_ex,
+    merge_partials, bwd_ex, bwd_workspace_size, accumulate), each following its C ABI
+    contract (outputs written into the buffers passed in) with the oracle's arithmetic,
+    so the driver's own buffer handling runs unchanged."""
+
+    def __init__(self):
+        self.calls = []
+
+    def fwd_ex(self, q, k, v, causal=False, scale=None, stream=None, **kw):
+        import oracle
+        self.calls.append("fwd_ex")
+        o, l = oracle.attention_forward(q.double().numpy(), k.double().numpy(), v.double().numpy(),
+                                        causal=causal, scale=scale)
+        return torch.from_numpy(o).to(q.dtype), torch.from_numpy(l).float()
+
+    def merge_partials(self, o_acc, lse_acc, o_part, lse_part, out=None, stream=None):
+        import numpy as np
+
+        import oracle
+        self.calls.append("merge_partials")
+        mo, ml = oracle.merge_partials(
+            np.stack([o_acc.double().numpy(), o_part.double().numpy()]),
+            np.stack([lse_acc.double().numpy().transpose(0, 2, 1),
+                      lse_part.double().numpy().transpose(0, 2, 1)]))
+        o_acc.copy_(torch.from_numpy(mo))
+        lse_acc.copy_(torch.from_numpy(ml.transpose(0, 2, 1)))
+        if out is not None:
+            out.copy_(o_acc)
+        return o_acc, lse_acc
+
+    def bwd_workspace_size(self, B, H, N, d):
+        return 256
+
+    def bwd_ex(self, q, k, v, out, dout, lse, causal=False, scale=None, dq=None, dk=None, dv=None,
+               workspace=None, stream=None, **kw):
+        import oracle
+        self.calls.append("bwd_ex")
+        assert dq is not None and dk is not None and dv is not None and workspace is not None
+        g = oracle.attention_backward_from_stats(*(t.double().numpy() for t in (q, k, v, out, dout, lse)),
+                                                 causal=causal, scale=scale)
+        for dst, src in zip((dq, dk, dv), g):
+            dst.copy_(torch.from_numpy(src))
+        return dq, dk, dv
+
+    def accumulate(self, acc, part=None, out=None, stream=None):
+        self.calls.append("accumulate")
+        assert part is not None or out is not None
+        if part is not None:
+            assert part.shape == acc.shape
+            acc += part.to(acc.dtype)
+        if out is not None:
+            assert out.shape == acc.shape
+            out.copy_(acc)
+        return acc
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulated_ring_through_the_binding_calls(world, causal, monkeypatch):
+    """The ring driver's real per-step code (_attend_and_merge, _grad_terms, _to_bf16)
+    against CPU stand-ins of the binding calls it makes: every result buffer is written
+    through those calls and the sums match the oracle over the whole sequence."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_155_b200 import ring
+    fake = _AbiStandIns()
+    for name in ("fwd_ex", "merge_partials", "bwd_ex", "bwd_workspace_size", "accumulate"):
+        monkeypatch.setattr(ring.ops, name, getattr(fake, name))
+    full = _full_inputs(world, seed=700 + world)
+    q, k, v, do = full
+    out, lse = ring.ring_attention_fwd_emulated(q, k, v, world, causal=causal, scale=0.6)
+    ref_o, ref_l = oracle.attention_forward(*[t.numpy() for t in full[:3]], causal=causal, scale=0.6)
+    np.testing.assert_allclose(out.numpy(), ref_o, atol=_ATOL)
+    np.testing.assert_allclose(lse.numpy(), ref_l, atol=_ATOL)
+    grads = ring.ring_attention_bwd_emulated(q, k, v, out, do, lse, world, causal=causal, scale=0.6)
+    refs = oracle.attention_backward(*[t.numpy() for t in full], causal=causal, scale=0.6)
+    for g, r in zip(grads, refs):
+        np.testing.assert_allclose(g.numpy(), r, atol=_ATOL)
+    pairs = world * world if not causal else world * (world + 1) // 2
+    assert fake.calls.count("bwd_ex") == pairs
+    # three sums per visited pair, plus one bf16 copy each of dK and dV per shard
+    assert fake.calls.count("accumulate") == 3 * pairs + 2 * world
