@@ -240,6 +240,30 @@ def timed_events(torch, fn, reps, flush=None):
     return statistics.median(times)
 
 
+def _barrier(world):
+    """Barrier over all ranks (no-op for one rank)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x, world, device):
+    """The largest of every rank's x (a device time: the job ends with its slowest rank)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank_step, steps, elapsed_ms):
+    """Whole-job rate: the units every rank processed over `steps` steps, divided by the
+    slowest rank's time (per-rank work is fixed as ranks are added: weak scaling)."""
+    return world * units_per_rank_step * steps / (elapsed_ms * 1e-3)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -277,15 +301,10 @@ def run_ours(args, rank, world, local_rank):
                    workspace=ws, main_events=(ev[2], ev[3]))
 
     def barrier():
-        if world > 1:
-            dist.barrier()
+        _barrier(world)
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return _max_over_ranks(x, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -313,7 +332,7 @@ def run_ours(args, rank, world, local_rank):
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
     bwd_main_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
     ms_per_step = elapsed_ms / K
-    value = world * f_step * K / (elapsed_ms * 1e-3) / 1e12
+    value = job_throughput(world, f_step, K, elapsed_ms) / 1e12
     status = fa.device_status()[0]
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -400,7 +419,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_ms = max_over_ranks(a.elapsed_time(b))
         h2d = sum(host[n].numel() * host[n].element_size() for n in host)
         d2h = sum(x.numel() * x.element_size() for x in (out, lse, dq, dk, dv))
-        e2e = {"value": world * f_step * Ke / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e2e = {"value": job_throughput(world, f_step, Ke, e2e_ms) / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e2e_ms / Ke, "steps": Ke,
                "pipelining": "2 device buffer sets; copy-in, compute and copy-out streams"}
