@@ -146,6 +146,26 @@ def test_varlen_sequences_are_independent():
             np.testing.assert_allclose(dk[cu[b]:cu[b + 1]].sum(axis=0), 0.0, atol=1e-12)
 
 
+def test_packing_example_of_the_long_text_page():
+    """The packing example of "ms-swift长文本训练优化，Flash-Attention显存省一半" (section on
+    --packing): a sample of 1024 tokens and one of 2048 are packed into one 3072-token
+    sequence instead of each being padded to max_length. Packed attention must give each
+    sample exactly its own attention (nothing crosses the boundary at token 1024), so
+    the packed forward equals the two separate forwards computed alone."""
+    lens = [1024, 2048]
+    cu = np.array([0, 1024, 3072], dtype=np.int64)
+    H, d = 1, 4
+    q, k, v = (_rand((3072, H, d), s) for s in (90, 91, 92))
+    out, lse = oracle.attention_forward_varlen(q, k, v, cu, causal=True, scale=0.5)
+    for b in range(2):
+        s0, s1 = cu[b], cu[b + 1]
+        o_b, l_b = oracle.attention_forward(q[None, s0:s1], k[None, s0:s1], v[None, s0:s1],
+                                            causal=True, scale=0.5)
+        np.testing.assert_allclose(out[s0:s1], o_b[0], rtol=0, atol=1e-13)
+        np.testing.assert_allclose(lse[:, s0:s1], l_b[0], rtol=0, atol=1e-13)
+    assert sum(lens) == 3072  # no padding tokens
+
+
 def test_window_pin_catches_planted_off_by_one(monkeypatch):
     q, k, v = _rand((1, 7, 1, 3), 80), _rand((1, 7, 1, 3), 81), _rand((1, 7, 1, 3), 82)
     orig = ref.window_mask
