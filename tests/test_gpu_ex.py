@@ -58,22 +58,26 @@ def test_qkvpacked_forward_and_backward(d, causal):
 
 
 LENS = [1, 127, 128, 129, 300, 0, 700, 5]
+# The packing example of the long-text ms-swift page: samples of 1024 and 2048 tokens
+# packed into one 3072-token batch.
+PAGE_PACKING = [1024, 2048]
 
 
+@pytest.mark.parametrize("lens", [LENS, PAGE_PACKING], ids=["ragged", "page_packing_example"])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d", [64, 128])
-def test_varlen_forward_and_backward(d, causal):
+def test_varlen_forward_and_backward(d, causal, lens):
     H = 2
-    cu = np.concatenate([[0], np.cumsum(LENS)]).astype(np.int32)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     total = int(cu[-1])
-    g = torch.Generator().manual_seed(9300 + d + int(causal))
+    g = torch.Generator().manual_seed(9300 + d + int(causal) + (0 if lens is LENS else 17))
     q, k, v, do = (bf16_randn((total, H, d), g) for _ in range(4))
     sc = default_scale(d)
     cu_t = torch.from_numpy(cu).cuda()
     qc, kc, vc, doc = (t.cuda() for t in (q, k, v, do))
-    out, lse = fa.fwd_ex(qc, kc, vc, causal=causal, scale=sc, cu_seqlens=cu_t, max_seqlen=max(LENS))
+    out, lse = fa.fwd_ex(qc, kc, vc, causal=causal, scale=sc, cu_seqlens=cu_t, max_seqlen=max(lens))
     grads = fa.bwd_ex(qc, kc, vc, out, doc, lse, causal=causal, scale=sc, cu_seqlens=cu_t,
-                      max_seqlen=max(LENS))
+                      max_seqlen=max(lens))
     torch.cuda.synchronize()
     assert fa.device_status()[0] == 0
     ref_o, ref_l = oracle.attention_forward_varlen(to_f64(q), to_f64(k), to_f64(v), cu,
