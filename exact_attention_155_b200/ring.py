@@ -14,7 +14,8 @@ The backward visits the shards in the same order. With the forward's output and 
 its query rows fixed, the recomputed backward of one (query shard, key/value shard)
 pair (fa_bwd_ex) gives that pair's terms of dQ, dK and dV, and each gradient is the sum
 of its terms (fa_accumulate keeps the sums in fp32). dQ stays on its rank; the sums
-for dK and dV travel with their key/value shard and reach its owner after a full turn.
+for dK and dV travel with their key/value shard and reach its owner after a full turn,
+each hop overlapping the next pair's backward.
 
 Every arithmetic step runs in the CUDA library; this module only orders calls and
 moves buffers (torch.distributed point-to-point, NCCL on GPUs).
@@ -74,13 +75,12 @@ def _attend_and_merge(q, k, v, mode, scale, o_acc, lse_acc, out, stream=None):
     ops.merge_partials(o_acc, lse_acc, o_p, lse_p, out=out, stream=stream)
 
 
-def _grad_terms(q, k, v, out, dout, lse, mode, scale, dq_acc, dk_acc, dv_acc, dq_out, bufs,
-                stream=None):
-    """Adds the terms of one (query shard, key/value shard) pair to the fp32 sums
-    dq_acc, dk_acc, dv_acc; writes the dQ sum as bf16 into `dq_out` when given. `bufs`
-    holds the bf16 term buffers and the backward workspace, made on first use."""
+def _pair_terms(q, k, v, out, dout, lse, mode, scale, bufs, stream=None):
+    """The terms of dQ, dK and dV of one (query shard, key/value shard) pair (bf16, in the
+    buffers of `bufs`, made on first use with the backward workspace), or None for a
+    skipped pair."""
     if mode == SKIP:
-        return
+        return None
     if not bufs:
         B, S, H, d = q.shape
         bufs["terms"] = tuple(torch.empty_like(q) for _ in range(3))
@@ -89,6 +89,15 @@ def _grad_terms(q, k, v, out, dout, lse, mode, scale, dq_acc, dk_acc, dv_acc, dq
     tq, tk, tv = bufs["terms"]
     ops.bwd_ex(q, k, v, out, dout, lse, causal=(mode == CAUSAL), scale=scale, dq=tq, dk=tk, dv=tv,
                workspace=bufs["ws"], stream=stream)
+    return bufs["terms"]
+
+
+def _add_terms(terms, dq_acc, dk_acc, dv_acc, dq_out, stream=None):
+    """Adds a pair's terms to the fp32 sums dq_acc, dk_acc, dv_acc (nothing for a skipped
+    pair); writes the dQ sum as bf16 into `dq_out` when given."""
+    if terms is None:
+        return
+    tq, tk, tv = terms
     ops.accumulate(dq_acc, tq, out=dq_out, stream=stream)
     ops.accumulate(dk_acc, tk, stream=stream)
     ops.accumulate(dv_acc, tv, stream=stream)
@@ -165,19 +174,26 @@ def ring_attention_bwd(q, k, v, out, dout, lse, causal: bool = False,
     sched = ring_schedule(rank, world, causal)
     last = last_step(sched)
     bufs = {}
+    dreqs = []  # the pass of the dK/dV sums started at the previous step
     for s, src, mode in sched:
         reqs = ring_pass(kv, nxt, rank, world, group) if s + 1 < world else []
-        _grad_terms(q, kv[0], kv[1], out, dout, lse, mode, scale, dq_acc, dkv[0], dkv[1],
-                    dq if s == last else None, bufs)
-        for r in reqs:
-            r.wait()
-        if world > 1:
-            # The dK/dV sums of the shard held now move on with it; after the last step
-            # this pass brings every rank the sums of its own shard.
-            for r in ring_pass(dkv, dkv_nxt, rank, world, group):
+        terms = _pair_terms(q, kv[0], kv[1], out, dout, lse, mode, scale, bufs)
+        # The sums of the shard held now arrive from rank - 1 while the terms are computed.
+        if dreqs:
+            for r in dreqs:
                 r.wait()
             dkv, dkv_nxt = dkv_nxt, dkv
+        _add_terms(terms, dq_acc, dkv[0], dkv[1], dq if s == last else None)
+        # They move on with their shard; after the last step this pass brings every rank
+        # the sums of its own shard.
+        dreqs = ring_pass(dkv, dkv_nxt, rank, world, group) if world > 1 else []
+        for r in reqs:
+            r.wait()
         kv, nxt = nxt, kv
+    for r in dreqs:
+        r.wait()
+    if dreqs:
+        dkv, dkv_nxt = dkv_nxt, dkv
     dk, dv = torch.empty_like(k), torch.empty_like(v)
     _to_bf16(dkv[0], dk)
     _to_bf16(dkv[1], dv)
@@ -209,8 +225,8 @@ def ring_attention_bwd_emulated(q, k, v, out, dout, lse, world: int, causal: boo
         sched = ring_schedule(rank, world, causal)
         last = last_step(sched)
         for s, src, mode in sched:
-            _grad_terms(qs, ks[src], vs[src], os_, dos, ls, mode, scale, dq_acc, dk_acc[src],
-                        dv_acc[src], dq if s == last else None, bufs)
+            terms = _pair_terms(qs, ks[src], vs[src], os_, dos, ls, mode, scale, bufs)
+            _add_terms(terms, dq_acc, dk_acc[src], dv_acc[src], dq if s == last else None)
         dqs.append(dq)
     dks, dvs = [], []
     for j in range(world):

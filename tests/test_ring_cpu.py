@@ -93,22 +93,30 @@ def _oracle_attend_and_merge(qs, ks, vs, mode, scale, o_acc, lse_acc, out, strea
         out.copy_(o_acc)
 
 
-def _oracle_grad_terms(qs, ks, vs, out, dout, lse, mode, scale, dq_acc, dk_acc, dv_acc, dq_out,
-                       bufs, stream=None):
-    """Stand-in for ring._grad_terms on CPU tensors: the oracle's terms of one shard
-    pair, added to the running sums."""
+def _oracle_pair_terms(qs, ks, vs, out, dout, lse, mode, scale, bufs, stream=None):
+    """Stand-in for ring._pair_terms on CPU tensors: the oracle's terms of one shard
+    pair (None for a skipped pair)."""
     import oracle
     from exact_attention_155_b200 import ring
-    _SEAM_CALLS.append(("bwd", mode, dq_out is not None))
+    _SEAM_CALLS.append(("terms", mode, False))
     if mode == ring.SKIP:
-        return
+        return None
     to64 = lambda t: t.double().numpy()
-    tq, tk, tv = oracle.attention_backward_from_stats(
+    g = oracle.attention_backward_from_stats(
         to64(qs), to64(ks), to64(vs), to64(out), to64(dout), to64(lse),
         causal=(mode == ring.CAUSAL), scale=scale)
-    dq_acc += torch.from_numpy(tq).to(dq_acc.dtype)
-    dk_acc += torch.from_numpy(tk).to(dk_acc.dtype)
-    dv_acc += torch.from_numpy(tv).to(dv_acc.dtype)
+    return tuple(torch.from_numpy(t) for t in g)
+
+
+def _oracle_add_terms(terms, dq_acc, dk_acc, dv_acc, dq_out, stream=None):
+    """Stand-in for ring._add_terms: adds the terms to the running sums."""
+    _SEAM_CALLS.append(("bwd", "skip" if terms is None else "pair", dq_out is not None))
+    if terms is None:
+        return
+    tq, tk, tv = terms
+    dq_acc += tq.to(dq_acc.dtype)
+    dk_acc += tk.to(dk_acc.dtype)
+    dv_acc += tv.to(dv_acc.dtype)
     if dq_out is not None:
         dq_out.copy_(dq_acc)
 
@@ -125,7 +133,8 @@ _ATOL = 1e-5
 
 def _use_oracle_seams(ring):
     ring._attend_and_merge = _oracle_attend_and_merge
-    ring._grad_terms = _oracle_grad_terms
+    ring._pair_terms = _oracle_pair_terms
+    ring._add_terms = _oracle_add_terms
     ring._to_bf16 = _oracle_to_bf16
 
 
@@ -263,7 +272,8 @@ def test_emulated_ring_fwd_and_bwd_on_cpu(world, causal, monkeypatch):
     import oracle
     from exact_attention_155_b200 import ring
     monkeypatch.setattr(ring, "_attend_and_merge", _oracle_attend_and_merge)
-    monkeypatch.setattr(ring, "_grad_terms", _oracle_grad_terms)
+    monkeypatch.setattr(ring, "_pair_terms", _oracle_pair_terms)
+    monkeypatch.setattr(ring, "_add_terms", _oracle_add_terms)
     monkeypatch.setattr(ring, "_to_bf16", _oracle_to_bf16)
     full = _full_inputs(world, seed=99 + world)
     q, k, v, do = full
@@ -387,7 +397,8 @@ class _AbiStandIns:
 @pytest.mark.parametrize("world", [1, 2, 3])
 @pytest.mark.parametrize("causal", [False, True])
 def test_emulated_ring_through_the_binding_calls(world, causal, monkeypatch):
-    """The ring driver's real per-step code (_attend_and_merge, _grad_terms, _to_bf16)
+    """The ring driver's real per-step code (_attend_and_merge, _pair_terms, _add_terms,
+    _to_bf16)
     against CPU stand-ins of the binding calls it makes: every result buffer is written
     through those calls and the sums match the oracle over the whole sequence."""
     import numpy as np
