@@ -129,14 +129,22 @@ def _device_ctx(device):
 _DEVICE_TYPE = "cuda"
 
 
+def _on_device_type(t: torch.Tensor) -> bool:
+    return t.is_cuda if _DEVICE_TYPE == "cuda" else t.device.type == _DEVICE_TYPE
+
+
 def _require(t: torch.Tensor, name: str, dtype=torch.bfloat16, shape=None, device=None):
     """Checks a tensor the library will read or write: a contiguous tensor of `dtype` on
     the library's device type, and, when given, exactly `shape` and on `device` (the
     kernels index every buffer from the sizes alone, so a wrong shape or another GPU's
-    buffer must never reach them)."""
+    buffer must never reach them). The passing case is one expression; the messages
+    are built only on failure."""
+    if (isinstance(t, torch.Tensor) and _on_device_type(t) and t.dtype == dtype and t.is_contiguous()
+            and (shape is None or t.shape == shape) and (device is None or t.device == device)):
+        return
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != _DEVICE_TYPE:
+    if not _on_device_type(t):
         raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype} (got {t.dtype}); inputs and outputs share one dtype")
@@ -144,8 +152,7 @@ def _require(t: torch.Tensor, name: str, dtype=torch.bfloat16, shape=None, devic
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} must have shape {tuple(shape)} (got {tuple(t.shape)})")
-    if device is not None and t.device != device:
-        raise ValueError(f"{name} must be on {device} like the other operands (got {t.device})")
+    raise ValueError(f"{name} must be on {device} like the other operands (got {t.device})")
 
 
 def _workspace(workspace, need: int, device):
@@ -238,7 +245,7 @@ def _row_stride(t: torch.Tensor, name: str, varlen: bool, shape, device=None) ->
     whose (H, d) block is contiguous; raises for any other layout."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
-    if t.device.type != _DEVICE_TYPE:
+    if not _on_device_type(t):
         raise ValueError(f"{name} must be a CUDA tensor (got {t.device})")
     if device is not None and t.device != device:
         raise ValueError(f"{name} must be on {device} like the other operands (got {t.device})")
