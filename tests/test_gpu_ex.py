@@ -210,3 +210,23 @@ def test_varlen_bench_size_sampled():
     _cmp_out(out[:, hs], lse[hs], ref_o, ref_l)
     refs = oracle.attention_backward_varlen(sub(q), sub(k), sub(v), sub(do), cu, causal=True, scale=sc)
     _cmp_grads(tuple(gr[:, hs] for gr in grads), refs)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_flash_attn_func_autograd(d, causal):
+    """The flash_attn-style entry point: out from the forward kernel, gradients from the
+    backward kernel through torch.autograd, against the oracle."""
+    B, N, H = 1, 300, 2
+    inp = make_inputs(B, N, H, d, 9700 + d + int(causal))
+    q, k, v = (inp[n].cuda().requires_grad_() for n in ("q", "k", "v"))
+    do = inp["dout"].cuda()
+    sc = default_scale(d)
+    out = fa.flash_attn_func(q, k, v, causal=causal)
+    out.backward(do)
+    torch.cuda.synchronize()
+    qf, kf, vf, dof = (to_f64(inp[n]) for n in ("q", "k", "v", "dout"))
+    ref_o, _ = oracle.attention_forward(qf, kf, vf, causal=causal, scale=sc)
+    assert np.max(np.abs(out.detach().float().cpu().numpy() - ref_o)) <= OUT_ATOL
+    refs = oracle.attention_backward(qf, kf, vf, dof, causal=causal, scale=sc)
+    _cmp_grads((q.grad, k.grad, v.grad), refs)
