@@ -235,3 +235,32 @@ def ring_attention_bwd_emulated(q, k, v, out, dout, lse, world: int, causal: boo
         _to_bf16(dk_acc[j], dks[j])
         _to_bf16(dv_acc[j], dvs[j])
     return torch.cat(dqs, dim=1), torch.cat(dks, dim=1), torch.cat(dvs, dim=1)
+
+
+class _RingAttention(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale, group):
+        out, lse = ring_attention_fwd(q, k, v, causal=causal, scale=scale, group=group)
+        ctx.save_for_backward(q, k, v, out, lse)
+        ctx.cfg = (causal, scale, group)
+        ctx.mark_non_differentiable(lse)
+        return out, lse
+
+    @staticmethod
+    def backward(ctx, dout, dlse):
+        q, k, v, out, lse = ctx.saved_tensors
+        causal, scale, group = ctx.cfg
+        dout = dout if dout.is_contiguous() else dout.contiguous()
+        dq, dk, dv = ring_attention_bwd(q, k, v, out, dout, lse, causal=causal, scale=scale,
+                                        group=group)
+        return dq, dk, dv, None, None, None
+
+
+def ring_flash_attn_func(q, k, v, causal: bool = False, softmax_scale: Optional[float] = None,
+                         group=None, return_lse: bool = False):
+    """Differentiable ring attention: this rank's shards q, k, v [B, S, H, d] (bf16) of a
+    sequence split into equal contiguous shards over the ranks of `group` (rank r holds
+    rows [r*S, (r+1)*S)). Returns this rank's rows of the output over the whole sequence,
+    or (out, lse); the backward runs ring_attention_bwd (every rank must call it)."""
+    out, lse = _RingAttention.apply(q, k, v, bool(causal), softmax_scale, group)
+    return (out, lse) if return_lse else out

@@ -422,3 +422,45 @@ def test_emulated_ring_through_the_binding_calls(world, causal, monkeypatch):
     assert fake.calls.count("bwd_ex") == pairs
     # three sums per visited pair, plus one bf16 copy each of dK and dV per shard
     assert fake.calls.count("accumulate") == 3 * pairs + 2 * world
+
+
+def _autograd_worker(rank, world, port, q):
+    """ring_flash_attn_func forward and autograd backward over gloo with the oracle
+    standing in for the kernels; returns this rank's output and input gradients."""
+    from exact_attention_155_b200 import ring
+
+    _use_oracle_seams(ring)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        full = _full_inputs(world, seed=808)
+        S = full[0].shape[1] // world
+        qs, ks, vs, dos = (t[:, rank * S:(rank + 1) * S].contiguous() for t in full)
+        for t in (qs, ks, vs):
+            t.requires_grad_()
+        out = ring.ring_flash_attn_func(qs, ks, vs, causal=True, softmax_scale=0.5)
+        out.backward(dos)
+        q.put((rank, out.detach().numpy(), [t.grad.numpy() for t in (qs, ks, vs)],
+               [t.numpy() for t in full]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_ring_flash_attn_func_autograd_over_gloo():
+    import numpy as np
+
+    import oracle
+    world = 2
+    got = _spawn(_autograd_worker, world)
+    full = got[0][2]
+    ref_o, _ = oracle.attention_forward(*full[:3], causal=True, scale=0.5)
+    refs = oracle.attention_backward(*full, causal=True, scale=0.5)
+    S = ref_o.shape[1] // world
+    for rank in range(world):
+        o, grads, _ = got[rank]
+        rows = slice(rank * S, (rank + 1) * S)
+        np.testing.assert_allclose(o, ref_o[:, rows], atol=_ATOL)
+        for g, r in zip(grads, refs):
+            np.testing.assert_allclose(g, r[:, rows], atol=_ATOL)
