@@ -22,9 +22,14 @@ __all__ = ["flash_attn_func", "flash_attn_qkvpacked_func", "flash_attn_varlen_fu
            "flash_attn_with_kvcache"]
 
 
-def _no_dropout(dropout_p):
+def _no_dropout(dropout_p, deterministic=False):
     if dropout_p:
         raise NotImplementedError("dropout_p must be 0: dropout is not part of this library")
+    if deterministic:
+        # The pages' flash_attn_func(..., deterministic=False) (MindSpore page, 常见问题与解决方案).
+        raise NotImplementedError("deterministic=True is not available: dQ is summed over key "
+                                  "tiles in a run-dependent order (dK and dV are bitwise "
+                                  "repeatable)")
 
 
 def _window(window_size, causal):
@@ -84,12 +89,12 @@ class _PackedAttention(torch.autograd.Function):
 
 def flash_attn_func(q, k, v, dropout_p: float = 0.0, softmax_scale: Optional[float] = None,
                     causal: bool = False, window_size: Tuple[int, int] = (-1, -1),
-                    return_attn_probs: bool = False):
+                    deterministic: bool = False, return_attn_probs: bool = False):
     """Exact attention of q, k, v [batch, seqlen, nheads, headdim] (bf16, CUDA); returns
     out [batch, seqlen, nheads, headdim], or (out, lse [batch, nheads, seqlen]) with
     return_attn_probs=True. softmax_scale=None is 1/sqrt(headdim); window_size=(left,
     right) limits query i to keys [i - left, i + right] (-1: unbounded)."""
-    _no_dropout(dropout_p)
+    _no_dropout(dropout_p, deterministic)
     out, lse = _Attention.apply(q, k, v, bool(causal), softmax_scale, _window(window_size, causal),
                                 None, None)
     return (out, lse) if return_attn_probs else out
@@ -97,10 +102,10 @@ def flash_attn_func(q, k, v, dropout_p: float = 0.0, softmax_scale: Optional[flo
 
 def flash_attn_qkvpacked_func(qkv, dropout_p: float = 0.0, softmax_scale: Optional[float] = None,
                               causal: bool = False, window_size: Tuple[int, int] = (-1, -1),
-                              return_attn_probs: bool = False):
+                              deterministic: bool = False, return_attn_probs: bool = False):
     """flash_attn_func on a packed qkv [batch, seqlen, 3, nheads, headdim], read in place;
     its gradient is packed the same way."""
-    _no_dropout(dropout_p)
+    _no_dropout(dropout_p, deterministic)
     out, lse = _PackedAttention.apply(qkv, bool(causal), softmax_scale, _window(window_size, causal))
     return (out, lse) if return_attn_probs else out
 
@@ -109,13 +114,13 @@ def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: in
                            max_seqlen_k: int, dropout_p: float = 0.0,
                            softmax_scale: Optional[float] = None, causal: bool = False,
                            window_size: Tuple[int, int] = (-1, -1),
-                           return_attn_probs: bool = False):
+                           deterministic: bool = False, return_attn_probs: bool = False):
     """Packed variable-length batches: q, k, v [total_tokens, nheads, headdim]; sequence b
     is tokens [cu_seqlens[b], cu_seqlens[b + 1]) (int32 on the device). Queries and keys
     share one packing (self-attention): cu_seqlens_k must be cu_seqlens_q and
     max_seqlen_k must equal max_seqlen_q. Returns out [total_tokens, nheads, headdim], or
     (out, lse [nheads, total_tokens])."""
-    _no_dropout(dropout_p)
+    _no_dropout(dropout_p, deterministic)
     if cu_seqlens_k is not cu_seqlens_q or int(max_seqlen_k) != int(max_seqlen_q):
         raise NotImplementedError("queries and keys must share one packing (pass the same "
                                   "cu_seqlens tensor for both, and equal max_seqlen)")

@@ -145,11 +145,14 @@ def test_varlen_uses_one_packing(fake):
         interface.flash_attn_varlen_func(q, k, v, cu, cu, 7, 8)
 
 
-def test_dropout_is_refused(fake):
+def test_dropout_and_deterministic_are_refused(fake):
     q, k, v = _qkv()
     with pytest.raises(NotImplementedError):
         interface.flash_attn_func(q, k, v, dropout_p=0.1)
-    assert fake.calls == []
+    with pytest.raises(NotImplementedError, match="deterministic"):
+        interface.flash_attn_func(q, k, v, deterministic=True)
+    interface.flash_attn_func(q, k, v, deterministic=False)  # the pages' setting
+    assert [c[0] for c in fake.calls] == ["fwd_ex"]
 
 
 def test_kvcache_step_routes_to_decode_and_paged_decode(fake):
