@@ -89,12 +89,18 @@ class _PackedAttention(torch.autograd.Function):
 
 def flash_attn_func(q, k, v, dropout_p: float = 0.0, softmax_scale: Optional[float] = None,
                     causal: bool = False, window_size: Tuple[int, int] = (-1, -1),
-                    deterministic: bool = False, return_attn_probs: bool = False):
+                    deterministic: bool = False, return_attn_probs: bool = False,
+                    block_size: Optional[int] = None):
     """Exact attention of q, k, v [batch, seqlen, nheads, headdim] (bf16, CUDA); returns
     out [batch, seqlen, nheads, headdim], or (out, lse [batch, nheads, seqlen]) with
     return_attn_probs=True. softmax_scale=None is 1/sqrt(headdim); window_size=(left,
-    right) limits query i to keys [i - left, i + right] (-1: unbounded)."""
+    right) limits query i to keys [i - left, i + right] (-1: unbounded). block_size (the
+    tiling hint of the ms-swift FA2/3 page's custom forward) is accepted and has no effect:
+    the kernels' tiles are fixed by the tensor-core shapes, and tiling does not change the
+    result of exact attention."""
     _no_dropout(dropout_p, deterministic)
+    if block_size is not None and int(block_size) <= 0:
+        raise ValueError("block_size must be positive")
     out, lse = _Attention.apply(q, k, v, bool(causal), softmax_scale, _window(window_size, causal),
                                 None, None)
     return (out, lse) if return_attn_probs else out

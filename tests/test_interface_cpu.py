@@ -167,3 +167,12 @@ def test_kvcache_step_routes_to_decode_and_paged_decode(fake):
     assert fake.calls[-1] == ("decode_paged", (2, 4), None) and lse.shape == (2, 3)
     with pytest.raises(ValueError):
         interface.flash_attn_with_kvcache(q, cache, cache)
+
+
+def test_block_size_hint_is_accepted_and_changes_nothing(fake):
+    q, k, v = _qkv(seed=9)
+    a = interface.flash_attn_func(q, k, v, causal=True, block_size=128)
+    b = interface.flash_attn_func(q, k, v, causal=True)
+    assert torch.equal(a, b)
+    with pytest.raises(ValueError):
+        interface.flash_attn_func(q, k, v, block_size=0)
