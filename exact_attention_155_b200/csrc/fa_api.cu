@@ -374,23 +374,18 @@ __global__ void timeout_probe_kernel(long long limit) {
 // Scratch for fa_bwd_noalloc, for callers that cannot allocate device memory: a
 // fixed-size array in the library's own device image (held by every GPU while the
 // library is loaded). Host code must not use the symbol as a pointer; the device
-// address is looked up per device with cudaGetSymbolAddress.
+// address is looked up with cudaGetSymbolAddress in the current context.
 static __device__ __align__(256) unsigned char g_bwd_noalloc_scratch[FA_BWD_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on device `dev` (resolved on first use, with
-// `dev` current: the caller's current device).
-fa_status noalloc_scratch(int dev, void** out) {
-  std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    cudaError_t e = cudaGetSymbolAddress(&ptr, g_bwd_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_fail(e, "fa_bwd_noalloc: cudaGetSymbolAddress(scratch)");
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+// Device address of the scratch array in the current device's context. Looked up on
+// every call (cudaGetSymbolAddress allocates nothing): the address belongs to the
+// context that loaded the library's device code, so a cached value would go stale if
+// the caller reset the device and a new primary context loaded the code elsewhere.
+fa_status noalloc_scratch(void** out) {
+  void* ptr = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&ptr, g_bwd_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_bwd_noalloc: cudaGetSymbolAddress(scratch)");
+  *out = ptr;
   return FA_OK;
 }
 
@@ -543,11 +538,10 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
                 "fa_bwd_noalloc: this problem needs %zu bytes of scratch but the built-in "
                 "scratch holds %u; call fa_bwd with a caller-provided workspace instead",
                 need, FA_BWD_NOALLOC_SCRATCH_BYTES);
-  int dev = 0;
-  fa_status st = current_device(&dev, nullptr);
+  fa_status st = current_device(nullptr, nullptr);
   if (st != FA_OK) return st;
   void* scratch = nullptr;
-  if ((st = noalloc_scratch(dev, &scratch)) != FA_OK) return st;
+  if ((st = noalloc_scratch(&scratch)) != FA_OK) return st;
   return fa_bwd(q, k, v, out, dout, lse, dq, dk, dv, B, H, N, d, causal, scale, scratch,
                 FA_BWD_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -57,6 +57,11 @@ __global__ void __launch_bounds__(256) merge_kernel(const MergeParams p) {
     }
 #pragma unroll
     for (int i = 0; i < 8; ++i) oa[i] = res[i];
+    // The row's TPR threads are consecutive lanes of one warp and all read lse_acc[li]
+    // above; the write waits until every one of them has.
+    const int lane = static_cast<int>(threadIdx.x & 31);
+    const unsigned row_mask = (TPR == 32 ? 0xffffffffu : ((1u << TPR) - 1u)) << (lane - sub);
+    __syncwarp(row_mask);
     if (sub == 0) p.lse_acc[li] = m + logf(wa + wp);
   }
   if (p.out != nullptr) {

@@ -123,13 +123,18 @@ def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: in
                            deterministic: bool = False, return_attn_probs: bool = False):
     """Packed variable-length batches: q, k, v [total_tokens, nheads, headdim]; sequence b
     is tokens [cu_seqlens[b], cu_seqlens[b + 1]) (int32 on the device). Queries and keys
-    share one packing (self-attention): cu_seqlens_k must be cu_seqlens_q and
-    max_seqlen_k must equal max_seqlen_q. Returns out [total_tokens, nheads, headdim], or
+    share one packing (self-attention): cu_seqlens_k must hold the same offsets as
+    cu_seqlens_q (the same tensor, or an equal copy) and max_seqlen_k must equal
+    max_seqlen_q. Returns out [total_tokens, nheads, headdim], or
     (out, lse [nheads, total_tokens])."""
     _no_dropout(dropout_p, deterministic)
-    if cu_seqlens_k is not cu_seqlens_q or int(max_seqlen_k) != int(max_seqlen_q):
-        raise NotImplementedError("queries and keys must share one packing (pass the same "
-                                  "cu_seqlens tensor for both, and equal max_seqlen)")
+    same = cu_seqlens_k is cu_seqlens_q or (
+        isinstance(cu_seqlens_k, torch.Tensor) and isinstance(cu_seqlens_q, torch.Tensor)
+        and cu_seqlens_k.shape == cu_seqlens_q.shape and cu_seqlens_k.device == cu_seqlens_q.device
+        and bool(torch.equal(cu_seqlens_k, cu_seqlens_q)))
+    if not same or int(max_seqlen_k) != int(max_seqlen_q):
+        raise NotImplementedError("queries and keys must share one packing (equal cu_seqlens "
+                                  "offsets for both, and equal max_seqlen)")
     out, lse = _Attention.apply(q, k, v, bool(causal), softmax_scale, _window(window_size, causal),
                                 cu_seqlens_q, int(max_seqlen_q))
     return (out, lse) if return_attn_probs else out

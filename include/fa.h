@@ -115,8 +115,9 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   dq, dk, dv         : [B, N, H, d] bf16 (written)
  *   workspace          : >= fa_bwd_workspace_size(B,H,N,d) bytes, 256-byte aligned;
  *                        contents on entry are ignored and left undefined.
- * The dq accumulation order across key tiles is not fixed (fp32 atomics), so dq
- * may differ in the last bits between runs; dk and dv are bitwise repeatable.
+ * dq is summed over key tiles with fp32 reductions into the workspace in an order
+ * that is not fixed, so dq may differ in the last bits between runs; dk and dv are
+ * bitwise repeatable.
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
@@ -167,9 +168,10 @@ fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out
  *    (fa_bwd_workspace_size) exceeds it are rejected with FA_ERR_WORKSPACE before
  *    anything is launched; use fa_bwd with your own workspace for those.
  *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating library routine.
- *  - The first call on each device looks up the scratch array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call before
- *    any stream capture.
+ *  - Every call looks up the scratch array's device address in the current
+ *    device's context (cudaGetSymbolAddress, which allocates nothing). The first
+ *    call on a device may load the library's device code there; make that first
+ *    call before any stream capture.
  *  - All calls on a device share the one scratch array, which keeps whatever the
  *    last call left in it (the backward re-initialises what it needs). Two calls
  *    whose executions overlap on the GPU (different streams, no ordering between

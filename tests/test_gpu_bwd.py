@@ -55,5 +55,5 @@ def test_bwd_dk_dv_are_deterministic():
     a = _run(inp, True, default_scale(128))
     b = _run(inp, True, default_scale(128))
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
-    # dq is accumulated with fp32 atomics; it must still agree to rounding.
+    # dq is summed with fp32 reductions in an order that is not fixed; it must still agree to rounding.
     assert torch.allclose(a[0].float(), b[0].float(), atol=1e-2, rtol=0)

@@ -139,8 +139,11 @@ def test_varlen_uses_one_packing(fake):
                                                causal=True)
     np.testing.assert_allclose(out.detach().numpy(), ref_o, atol=1e-12)
     assert fake.calls[0] == ("fwd_ex", True, None, None, True, 7)
+    # An equal copy of the offsets is the same packing.
+    again = interface.flash_attn_varlen_func(q, k, v, cu, cu.clone(), 7, 7, causal=True)
+    np.testing.assert_allclose(again.detach().numpy(), ref_o, atol=1e-12)
     with pytest.raises(NotImplementedError):
-        interface.flash_attn_varlen_func(q, k, v, cu, cu.clone(), 7, 7)
+        interface.flash_attn_varlen_func(q, k, v, cu, torch.tensor([0, 4, 10], dtype=torch.int32), 7, 7)
     with pytest.raises(NotImplementedError):
         interface.flash_attn_varlen_func(q, k, v, cu, cu, 7, 8)
 
