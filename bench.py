@@ -47,18 +47,15 @@ STEPS5 = dict(B=2, H=16, d=64, Ncap=2048, steps=100)
 TINY = dict(B=1, H=2, N=128, d=64)
 VIT = dict(B=2, H=16, N=1024, d=64)
 
-# DRAM bytes per launch of the backward main kernel from an ncu capture, valid only
-# for the kernel source it was taken on (sha256 of csrc/bwd.cuh).
+
 # Nominal B200 figures the targets are stated against (dense bf16, HBM3e): reported
 # beside the measured-peak fractions.
 NOMINAL_TFLOPS = 2250.0
 NOMINAL_HBM_GBS = 8000.0
 
-# Throughput of cp.reduce.async.bulk .add.f32 from shared memory into a 256 MiB fp32
-# buffer, all SMs reducing 16 KB chunks (independent of 2, 4 or 8 chunks in flight per SM),
-# measured on this machine type by exact_attention_155_b200/csrc/l2_reduction_rate.cu.
-L2_REDUCTION_GBS = 3840.0
-
+# DRAM bytes per launch of the backward main kernel from an ncu capture of the training
+# workload, valid only for the kernel source it was taken on (sha256 of csrc/bwd.cuh);
+# null otherwise.
 BWD_TRAFFIC = {"src_sha256": "00ade1531fe1e214ba9fdbe8ae5ee1f1bf2a53490bebce85486bcab486fb1ad7",
                "bytes_per_launch": 828.82e6 + 509.35e6}
 
@@ -354,18 +351,6 @@ def run_ours(args, rank, world, local_rank):
                 "sm_mhz_median": clocks["sm_mhz"] if clocks else None,
                 "traffic": traffic, "avg_launch_ms": bwd_main_ms,
                 "algorithmic_flop_per_launch": f_bwd}
-    # The backward's other bound: every (key tile, visible query tile) pair adds a
-    # 128 x d fp32 block of dQ into the L2-resident accumulator with a bulk reduction.
-    nkt = (w["N"] + 127) // 128
-    pairs = nkt * (nkt + 1) // 2 if w["causal"] else nkt * nkt
-    red_bytes = float(pairs) * 128 * w["d"] * 4 * w["B"] * w["H"]
-    roofline["l2_reduction"] = {
-        "bytes_per_launch": red_bytes,
-        "achieved_gbs": red_bytes / (bwd_main_ms * 1e-3) / 1e9,
-        "peak_gbs": L2_REDUCTION_GBS,
-        "frac": red_bytes / (bwd_main_ms * 1e-3) / 1e9 / L2_REDUCTION_GBS,
-        "peak_kind": "bulk fp32 reduction rate measured by csrc/l2_reduction_rate.cu (all SMs, "
-                     "16.8 B/clk/SM into a 256 MiB buffer); not one of the peaks in MEASURED_PEAKS.json"}
 
     # ---- end to end through the public API from pinned host buffers
     # Every step copies its own inputs host->device and its results device->host.

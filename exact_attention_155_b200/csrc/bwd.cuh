@@ -26,6 +26,9 @@
 //    d = 128, vector atomics for d = 64); warp 12 issues TMA; warp 13 issues
 //    tcgen05.mma.
 //  * bwd_dq_convert_kernel: dq = bf16(accumulator).
+// The fp32 reductions of dQ land in an order that is not fixed, so dQ may differ in
+// its last bits between runs. bwd_det.cuh has the bitwise-repeatable alternative
+// (separate dK/dV and dQ kernels, seven tile products per tile pair instead of five).
 #pragma once
 
 #include <math.h>
@@ -37,7 +40,7 @@ namespace fa {
 struct BwdParams {
   int B, H, N, Np;      // N: sequence length (dense) or the largest one (variable length);
                         // Np = N rounded up to a multiple of 128
-  int nqt;              // Np / 128
+  int nqt;              // Np / 128: key tiles and query tiles per (batch, head)
   int head_group;       // heads scheduled together (divides B*H), for L2 reuse
   int window_left;      // keys visible to query i: [i - window_left, i + window_right],
   int window_right;     // -1 = unbounded on that side (causal: window_right = 0)
@@ -50,7 +53,7 @@ struct BwdParams {
   const uint16_t* out;  // forward output
   const uint16_t* dout;
   const float* lse;     // dense [B, H, N]; variable [H, total]; natural log
-  float* dq_acc;        // [B, H, Np, d] fp32
+  float* dq_acc;        // [B, H, Np, d] fp32 (fused kernel only; null for bwd_det.cuh)
   float* lse2;          // [B, H, Np] log2 units (+inf on rows past the sequence)
   float* dvec;          // [B, H, Np] rowsum(dO * O)
   uint16_t* dq;
@@ -64,6 +67,9 @@ enum : unsigned int {
   kSiteBwdSoftmax = 0x203,
   kSiteBwdDrain = 0x204,
   kSiteBwdSeqlens = 0x205,
+  kSiteBwdQProducer = 0x211,
+  kSiteBwdQMma = 0x212,
+  kSiteBwdQSoftmax = 0x213,
   kSiteBwdSmemAlign = 0x2FF
 };
 
@@ -136,9 +142,11 @@ __global__ void __launch_bounds__(256) bwd_pre_kernel(const BwdParams p) {
     p.dvec[row] = real ? acc : 0.f;
     p.lse2[row] = lse;
   }
-  float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D + sub * 8);
-  z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-  z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.dq_acc != nullptr) {  // the fused kernel's fp32 dQ accumulator
+    float4* z = reinterpret_cast<float4*>(p.dq_acc + row * D + sub * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 template <int D>
@@ -205,13 +213,6 @@ struct BwdLayout {
   static_assert(kBytes <= 232448, "shared memory budget");
 };
 
-// Of every 16 exponential pairs of the P pass, this many use the FMA-pipe polynomial
-// (exp2_poly2) instead of the MUFU unit.
-#ifndef FA_BWD_POLY_PAIRS
-#define FA_BWD_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairsBwd = FA_BWD_POLY_PAIRS;
-
 
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
@@ -241,9 +242,6 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
                : "memory");
 }
-
-// Trace slot of (role, iteration, event) for the traced CTA (block 0).
-#define FA_BWD_TR(role, n, e) ((((role) * 128 + ((n) & 127)) * 8) + (e))
 
 // GENERAL = false compiles the plain dense case (no sequence offsets, no window,
 // CAUSAL fixed); GENERAL = true reads the window and cu_seqlens at run time.
@@ -345,7 +343,6 @@ __global__ void __launch_bounds__(448, 1)
         const int s = n % L::kQStages;
         if (!wait_bar(BAR(L::kQEmpty + s), ((n / L::kQStages) & 1) ^ 1u, abort_flag, kSiteBwdProducer))
           break;
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(3, n, 0));
         const uint32_t sQ = base + L::kQ0 + s * L::kTile;
         mbar_arrive_expect_tx(BAR(L::kQFull + s), L::kTile + 1024);
         for (int bx = 0; bx < D / 64; ++bx)
@@ -355,7 +352,6 @@ __global__ void __launch_bounds__(448, 1)
         bulk_load(sv + 512, dvec_h + it * 128, 512, BAR(L::kQFull + s));
         ++nq;
         if (!wait_bar(BAR(L::kDOEmpty), (n & 1) ^ 1u, abort_flag, kSiteBwdProducer)) break;
-        FA_TRACE_EVENT(blockIdx.x == 0, FA_BWD_TR(3, n, 1));
         mbar_arrive_expect_tx(BAR(L::kDOFull), L::kTile);
         for (int bx = 0; bx < D / 64; ++bx)
           tma_load_4d(base + L::kDO + bx * 16384, &tmdO, BAR(L::kDOFull), bx * 64, h, trow + it * 128, tb);
@@ -410,7 +406,6 @@ __global__ void __launch_bounds__(448, 1)
         if (n > 0) {
           if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDQFree), (n - 1) & 1, abort_flag, kSiteBwdMma)))) break;
         }
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 0));
         if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDOFull), n & 1, abort_flag, kSiteBwdMma)))) break;
         tc_fence_after();
 #pragma unroll
@@ -420,17 +415,14 @@ __global__ void __launch_bounds__(448, 1)
                   kk > 0 ? 1u : 0u);
         }
         umma_commit_w(BAR(L::kDPFull));
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 1));
         // dV += P^T dO_n
         if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kPFull), n & 1, abort_flag, kSiteBwdMma)))) break;
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 2));
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           umma_ts_w(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
                   (n > 0 || kk > 0) ? 1u : 0u);
         umma_commit_w(BAR(L::kDOEmpty));
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 3));
         // S^T(n+1): the S columns are free once dV(n) (issued above, executed in order)
         // has read P(n); the dS pass keeps P(n) in registers.
         if (n + 1 < niter) {
@@ -440,10 +432,8 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
           issue_st(n + 1);
         }
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 4));
         if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDSFull), n & 1, abort_flag, kSiteBwdMma)))) break;
         tc_fence_after();
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 5));
         // dQ_n first, so the drain reads it out of TMEM while dK(n) runs.
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
@@ -462,7 +452,6 @@ __global__ void __launch_bounds__(448, 1)
                   sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdKV, (n > 0 || kk > 0) ? 1u : 0u);
         umma_commit_w(BAR(L::kDSFree));
         umma_commit_w(BAR(L::kQEmpty + s));
-        FA_TRACE_EVENT(blockIdx.x == 0 && lane == 0, FA_BWD_TR(0, n, 6));
       }
       if (ok) umma_commit_w(BAR(L::kMmaDone));
       umma_commit_w(BAR(L::kDrain));
@@ -479,7 +468,6 @@ __global__ void __launch_bounds__(448, 1)
     const bool key_ok = key < seqlen;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float sl2 = p.scale_log2;
-    [[maybe_unused]] const bool tr = blockIdx.x == 0 && threadIdx.x == 0;  // traced thread
     bool ok = true;
     for (int n = 0; n < niter; ++n) {
       const int it = it0 + n;
@@ -489,7 +477,6 @@ __global__ void __launch_bounds__(448, 1)
       if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kQFull + s), (n / L::kQStages) & 1,
                                                    abort_flag, kSiteBwdSoftmax));
       if (!ok) break;
-      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 0));
       tc_fence_after();
       uint32_t s0[32], s1[32];
       tmem_ld32(tS + lane_off + c0, s0);
@@ -501,7 +488,6 @@ __global__ void __launch_bounds__(448, 1)
         tc_fence_before();
         mbar_arrive(BAR(L::kSLoaded + wq));
       }
-      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 1));
       // Local columns c in [qlo_c, qhi_c] are the queries that see this key (window
       // [key - wr, key + wl]); none if the key is past the sequence. Queries past the
       // sequence have lse2 = +inf, so their P is already 0.
@@ -513,14 +499,8 @@ __global__ void __launch_bounds__(448, 1)
       for (int c2 = 0; c2 < 32; ++c2) {
         const int c = 2 * c2;
         const uint32_t* src = c < 32 ? s0 : s1;
-        float e0 = __uint_as_float(src[c & 31]) * sl2 - vec[c];
-        float e1 = __uint_as_float(src[(c + 1) & 31]) * sl2 - vec[c + 1];
-        if ((c2 & 15) < kPolyPairsBwd) {
-          exp2_poly2(e0, e1);  // FMA/ALU pipes
-        } else {
-          e0 = ex2_approx(e0);  // MUFU
-          e1 = ex2_approx(e1);
-        }
+        const float e0 = ex2_approx(__uint_as_float(src[c & 31]) * sl2 - vec[c]);
+        const float e1 = ex2_approx(__uint_as_float(src[(c + 1) & 31]) * sl2 - vec[c + 1]);
         const float p0 = (c < qlo_c || c > qhi_c) ? 0.f : e0;
         const float p1 = (c + 1 < qlo_c || c + 1 > qhi_c) ? 0.f : e1;
         pk[c2] = pack_bf16x2(p0, p1);
@@ -539,13 +519,11 @@ __global__ void __launch_bounds__(448, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(L::kPFull));
-      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 2));
 
       ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDPFull), n & 1, abort_flag, kSiteBwdSoftmax));
       if (ok && n > 0)
         ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDSFree), (n - 1) & 1, abort_flag, kSiteBwdSoftmax));
       if (!ok) break;
-      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 3));
       tc_fence_after();
       const float* dvec = vec + 128;
       uint32_t dp0[32], dp1[32];
@@ -579,7 +557,6 @@ __global__ void __launch_bounds__(448, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(BAR(L::kDSFull));
-      FA_TRACE_EVENT(tr, FA_BWD_TR(1, n, 4));
     }
     if (ok) ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kMmaDone), 0, abort_flag, kSiteBwdSoftmax));
     if (ok) {
@@ -620,7 +597,6 @@ __global__ void __launch_bounds__(448, 1)
       // All four drain warps leave together: they share named barriers below.
       ok = named_bar_and(1, 128, ok);
       if (!ok) break;
-      FA_TRACE_EVENT(blockIdx.x == 0 && threadIdx.x == 256, FA_BWD_TR(2, n, 0));
       tc_fence_after();
       if constexpr (D == 128) {
         // Read all of dQ^T (128 queries for this thread's head-dim index r), free the
@@ -639,7 +615,6 @@ __global__ void __launch_bounds__(448, 1)
         reg_fence32(o3);
         tc_fence_before();
         mbar_arrive(BAR(L::kDQFree));
-        FA_TRACE_EVENT(blockIdx.x == 0 && threadIdx.x == 256, FA_BWD_TR(2, n, 1));
         float* gtile = p.dq_acc + (static_cast<size_t>(bh) * p.Np + static_cast<size_t>(it) * 128) * D;
         const bool leader = (warp == 8 && lane == 0);
 #pragma unroll
@@ -657,7 +632,6 @@ __global__ void __launch_bounds__(448, 1)
             bulk_commit();
           }
         }
-        FA_TRACE_EVENT(blockIdx.x == 0 && threadIdx.x == 256, FA_BWD_TR(2, n, 2));
         continue;
       } else {
         const int qrow = it * 128 + r;

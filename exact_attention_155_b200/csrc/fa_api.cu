@@ -16,13 +16,14 @@
 #include "ptx.cuh"
 #include "fwd.cuh"
 #include "bwd.cuh"
+#include "bwd_det.cuh"
 #include "decode.cuh"
 #include "merge.cuh"
 #include "accumulate.cuh"
 
 namespace {
 
-constexpr int kAbiVersion = 1;
+constexpr int kAbiVersion = 2;
 thread_local std::string g_last_error;
 
 fa_status fail(fa_status st, const char* fmt, ...) {
@@ -193,6 +194,27 @@ fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CU
   return check_launch("fa_bwd main kernel launch");
 }
 
+template <int D, bool CAUSAL, bool GENERAL>
+fa_status launch_bwd_det(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                             const CUtensorMap& mdo, fa::BwdParams p, int dev, cudaStream_t stream) {
+  using LA = fa::BwdKVLayout<D>;
+  using LB = fa::BwdQLayout<D>;
+  auto ka = fa::bwd_dkdv_kernel<D, CAUSAL, GENERAL>;
+  auto kb = fa::bwd_dq_kernel<D, CAUSAL, GENERAL>;
+  fa_status st = set_smem(ka, LA::kBytes, dev);
+  if (st != FA_OK) return st;
+  if ((st = set_smem(kb, LB::kBytes, dev)) != FA_OK) return st;
+  const unsigned grid = static_cast<unsigned>(p.nqt) * p.B * p.H;
+  // dK/dV: four heads per group (their Q and dO, 4 x 8 MiB at N = 16384, stay in L2).
+  p.head_group = head_group_for(p.B * p.H, 4);
+  ka<<<grid, LA::kThreads, LA::kBytes, stream>>>(mq, mk, mv, mdo, p);
+  if ((st = check_launch("fa_bwd dK/dV kernel launch")) != FA_OK) return st;
+  // dQ: eight heads per group (their K and V, 8 x 8 MiB at N = 16384, stay in L2).
+  p.head_group = head_group_for(p.B * p.H, 8);
+  kb<<<grid, LB::kThreads, LB::kBytes, stream>>>(mq, mk, mv, mdo, p);
+  return check_launch("fa_bwd dQ kernel launch");
+}
+
 // Strides (elements between consecutive tokens) of the eight row-major operands of a
 // backward call, in the order q, k, v, out, dout, dq, dk, dv.
 struct BwdStrides {
@@ -202,8 +224,8 @@ struct BwdStrides {
 fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                   const float* lse, void* dq, void* dk, void* dv, const RowLayout& lay,
                   const BwdStrides& rs, int wl, int wr, float scale, void* workspace,
-                  const fa::BwdWorkspace& ws, int dev, cudaStream_t stream, cudaEvent_t ev_start,
-                  cudaEvent_t ev_stop) {
+                  const fa::BwdWorkspace& ws, bool deterministic, int dev, cudaStream_t stream,
+                  cudaEvent_t ev_start, cudaEvent_t ev_stop) {
   const int B = lay.B, H = lay.H, N = lay.N, d = lay.d;
   CUtensorMap mq, mk, mv, mdo;
   fa_status st;
@@ -234,7 +256,8 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   p.dout = static_cast<const uint16_t*>(dout);
   p.lse = lse;
   char* w = static_cast<char*>(workspace);
-  p.dq_acc = reinterpret_cast<float*>(w + ws.dq_off);
+  // The deterministic kernels write dq directly: no fp32 accumulator to zero or convert.
+  p.dq_acc = deterministic ? nullptr : reinterpret_cast<float*>(w + ws.dq_off);
   p.lse2 = reinterpret_cast<float*>(w + ws.lse2_off);
   p.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
   p.dq = static_cast<uint16_t*>(dq);
@@ -250,6 +273,20 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   if (ev_start && (e = cudaEventRecord(ev_start, stream)) != cudaSuccess)
     return cuda_fail(e, "fa_bwd_profiled: record start event");
   const bool general = lay.cu_seqlens != nullptr || wl >= 0 || wr > 0;
+  if (deterministic) {
+    if (d == 64)
+      st = general ? launch_bwd_det<64, false, true>(mq, mk, mv, mdo, p, dev, stream)
+           : wr == 0 ? launch_bwd_det<64, true, false>(mq, mk, mv, mdo, p, dev, stream)
+                     : launch_bwd_det<64, false, false>(mq, mk, mv, mdo, p, dev, stream);
+    else
+      st = general ? launch_bwd_det<128, false, true>(mq, mk, mv, mdo, p, dev, stream)
+           : wr == 0 ? launch_bwd_det<128, true, false>(mq, mk, mv, mdo, p, dev, stream)
+                     : launch_bwd_det<128, false, false>(mq, mk, mv, mdo, p, dev, stream);
+    if (st != FA_OK) return st;
+    if (ev_stop && (e = cudaEventRecord(ev_stop, stream)) != cudaSuccess)
+      return cuda_fail(e, "fa_bwd_profiled: record stop event");
+    return FA_OK;
+  }
   if (d == 64)
     st = general ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, dev, stream)
          : wr == 0 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, dev, stream)
@@ -483,15 +520,15 @@ fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const voi
   const long long rs = static_cast<long long>(H) * d;
   const BwdStrides strides{rs, rs, rs, rs, rs, rs, rs, rs};
   return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, lay, strides, -1, causal ? 0 : -1, scale,
-                 workspace, ws, dev, static_cast<cudaStream_t>(stream),
+                 workspace, ws, false, dev, static_cast<cudaStream_t>(stream),
                  static_cast<cudaEvent_t>(main_start), static_cast<cudaEvent_t>(main_stop));
 }
 
 fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
                     const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens,
                     int total_tokens, int B, int H, int N, int d, const long long* row_strides,
-                    int causal, int window_left, int window_right, float scale, void* workspace,
-                    size_t workspace_bytes, void* stream) {
+                    int causal, int window_left, int window_right, float scale, int deterministic,
+                    void* workspace, size_t workspace_bytes, void* stream) {
   if (!row_strides) return fail(FA_ERR_INVALID_ARG, "fa_bwd_ex: row_strides is null");
   RowLayout lay;
   int wr = -1;
@@ -514,7 +551,7 @@ fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out
   const BwdStrides strides{row_strides[0], row_strides[1], row_strides[2], row_strides[3],
                            row_strides[4], row_strides[5], row_strides[6], row_strides[7]};
   return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, lay, strides, window_left, wr, scale, workspace,
-                 ws, dev, static_cast<cudaStream_t>(stream), nullptr, nullptr);
+                 ws, deterministic != 0, dev, static_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,

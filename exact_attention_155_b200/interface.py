@@ -22,14 +22,9 @@ __all__ = ["flash_attn_func", "flash_attn_qkvpacked_func", "flash_attn_varlen_fu
            "flash_attn_with_kvcache"]
 
 
-def _no_dropout(dropout_p, deterministic=False):
+def _no_dropout(dropout_p):
     if dropout_p:
         raise NotImplementedError("dropout_p must be 0: dropout is not part of this library")
-    if deterministic:
-        # The pages' flash_attn_func(..., deterministic=False) (MindSpore page, 常见问题与解决方案).
-        raise NotImplementedError("deterministic=True is not available: dQ is summed over key "
-                                  "tiles in a run-dependent order (dK and dV are bitwise "
-                                  "repeatable)")
 
 
 def _window(window_size, causal):
@@ -51,11 +46,11 @@ def _dense(t):
 
 class _Attention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, causal, scale, window, cu_seqlens, max_seqlen):
+    def forward(ctx, q, k, v, causal, scale, window, cu_seqlens, max_seqlen, deterministic):
         out, lse = ops.fwd_ex(q, k, v, causal=causal, scale=scale, window=window,
                               cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)
         ctx.save_for_backward(q, k, v, out, lse)
-        ctx.cfg = (causal, scale, window, cu_seqlens, max_seqlen)
+        ctx.cfg = (causal, scale, window, cu_seqlens, max_seqlen, deterministic)
         ctx.mark_non_differentiable(lse)
         return out, lse
 
@@ -63,28 +58,29 @@ class _Attention(torch.autograd.Function):
     def backward(ctx, dout, dlse):
         # lse is an output for inspection only (not differentiable).
         q, k, v, out, lse = ctx.saved_tensors
-        causal, scale, window, cu_seqlens, max_seqlen = ctx.cfg
+        causal, scale, window, cu_seqlens, max_seqlen, deterministic = ctx.cfg
         dq, dk, dv = ops.bwd_ex(q, k, v, out, _dense(dout), lse, causal=causal, scale=scale,
-                                window=window, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen)
-        return dq, dk, dv, None, None, None, None, None
+                                window=window, cu_seqlens=cu_seqlens, max_seqlen=max_seqlen,
+                                deterministic=deterministic)
+        return dq, dk, dv, None, None, None, None, None, None
 
 
 class _PackedAttention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, qkv, causal, scale, window):
+    def forward(ctx, qkv, causal, scale, window, deterministic):
         out, lse = ops.fwd_qkvpacked(qkv, causal=causal, scale=scale, window=window)
         ctx.save_for_backward(qkv, out, lse)
-        ctx.cfg = (causal, scale, window)
+        ctx.cfg = (causal, scale, window, deterministic)
         ctx.mark_non_differentiable(lse)
         return out, lse
 
     @staticmethod
     def backward(ctx, dout, dlse):
         qkv, out, lse = ctx.saved_tensors
-        causal, scale, window = ctx.cfg
+        causal, scale, window, deterministic = ctx.cfg
         dqkv = ops.bwd_qkvpacked(qkv, out, _dense(dout), lse, causal=causal, scale=scale,
-                                 window=window)
-        return dqkv, None, None, None
+                                 window=window, deterministic=deterministic)
+        return dqkv, None, None, None, None
 
 
 def flash_attn_func(q, k, v, dropout_p: float = 0.0, softmax_scale: Optional[float] = None,
@@ -97,12 +93,14 @@ def flash_attn_func(q, k, v, dropout_p: float = 0.0, softmax_scale: Optional[flo
     right) limits query i to keys [i - left, i + right] (-1: unbounded). block_size (the
     tiling hint of the ms-swift FA2/3 page's custom forward) is accepted and has no effect:
     the kernels' tiles are fixed by the tensor-core shapes, and tiling does not change the
-    result of exact attention."""
-    _no_dropout(dropout_p, deterministic)
+    result of exact attention. deterministic=True (the flag the MindSpore page's
+    常见问题与解决方案 sets) makes the backward bitwise repeatable (a slower kernel pair
+    that writes every gradient element once); the forward is repeatable either way."""
+    _no_dropout(dropout_p)
     if block_size is not None and int(block_size) <= 0:
         raise ValueError("block_size must be positive")
     out, lse = _Attention.apply(q, k, v, bool(causal), softmax_scale, _window(window_size, causal),
-                                None, None)
+                                None, None, bool(deterministic))
     return (out, lse) if return_attn_probs else out
 
 
@@ -111,8 +109,9 @@ def flash_attn_qkvpacked_func(qkv, dropout_p: float = 0.0, softmax_scale: Option
                               deterministic: bool = False, return_attn_probs: bool = False):
     """flash_attn_func on a packed qkv [batch, seqlen, 3, nheads, headdim], read in place;
     its gradient is packed the same way."""
-    _no_dropout(dropout_p, deterministic)
-    out, lse = _PackedAttention.apply(qkv, bool(causal), softmax_scale, _window(window_size, causal))
+    _no_dropout(dropout_p)
+    out, lse = _PackedAttention.apply(qkv, bool(causal), softmax_scale, _window(window_size, causal),
+                                      bool(deterministic))
     return (out, lse) if return_attn_probs else out
 
 
@@ -127,7 +126,7 @@ def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: in
     cu_seqlens_q (the same tensor, or an equal copy) and max_seqlen_k must equal
     max_seqlen_q. Returns out [total_tokens, nheads, headdim], or
     (out, lse [nheads, total_tokens])."""
-    _no_dropout(dropout_p, deterministic)
+    _no_dropout(dropout_p)
     same = cu_seqlens_k is cu_seqlens_q or (
         isinstance(cu_seqlens_k, torch.Tensor) and isinstance(cu_seqlens_q, torch.Tensor)
         and cu_seqlens_k.shape == cu_seqlens_q.shape and cu_seqlens_k.device == cu_seqlens_q.device
@@ -136,7 +135,7 @@ def flash_attn_varlen_func(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: in
         raise NotImplementedError("queries and keys must share one packing (equal cu_seqlens "
                                   "offsets for both, and equal max_seqlen)")
     out, lse = _Attention.apply(q, k, v, bool(causal), softmax_scale, _window(window_size, causal),
-                                cu_seqlens_q, int(max_seqlen_q))
+                                cu_seqlens_q, int(max_seqlen_q), bool(deterministic))
     return (out, lse) if return_attn_probs else out
 
 

@@ -42,7 +42,7 @@ _SIGNATURES = {
     "fa_bwd_ex": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                            _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int,
                            _c_int, _c_int, ctypes.POINTER(_c_ll), _c_int, _c_int, _c_int,
-                           _c_float, _c_void_p, _c_size_t, _c_void_p]),
+                           _c_float, _c_int, _c_void_p, _c_size_t, _c_void_p]),
     "fa_bwd_workspace_size": (_c_size_t, [_c_int, _c_int, _c_int, _c_int]),
     "fa_bwd": (_c_int, [_c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p, _c_void_p,
                         _c_void_p, _c_void_p, _c_void_p, _c_int, _c_int, _c_int, _c_int, _c_int,
@@ -324,8 +324,11 @@ def fwd_ex(q, k, v, causal: bool = False, scale: Optional[float] = None, window=
 def bwd_ex(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float] = None,
            window=None, cu_seqlens: Optional[torch.Tensor] = None,
            max_seqlen: Optional[int] = None, dq=None, dk=None, dv=None, workspace=None,
-           stream=None):
-    """Backward of fwd_ex (fa_bwd_ex): same layouts and options. Returns (dq, dk, dv)."""
+           stream=None, deterministic: bool = False):
+    """Backward of fwd_ex (fa_bwd_ex): same layouts and options. Returns (dq, dk, dv).
+
+    deterministic=True selects the bitwise-repeatable backward (separate dK/dV and dQ
+    kernels, no reductions into a shared accumulator); it is slower."""
     if not isinstance(q, torch.Tensor):
         raise TypeError("q must be a torch.Tensor")
     dev = q.device
@@ -344,8 +347,8 @@ def bwd_ex(q, k, v, out, dout, lse, causal: bool = False, scale: Optional[float]
     with _device_ctx(dev):
         _check(lib.fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(dout), _ptr(lse),
                              _ptr(dq), _ptr(dk), _ptr(dv), _ptr(cu_seqlens), total, B, H, N, d, rs,
-                             int(bool(causal)), wl, wr, _scale(scale, d), _ptr(workspace),
-                             workspace.numel(), _stream(stream)))
+                             int(bool(causal)), wl, wr, _scale(scale, d), int(bool(deterministic)),
+                             _ptr(workspace), workspace.numel(), _stream(stream)))
     return dq, dk, dv
 
 
@@ -361,7 +364,7 @@ def fwd_qkvpacked(qkv, causal: bool = False, scale: Optional[float] = None, wind
 
 
 def bwd_qkvpacked(qkv, out, dout, lse, causal: bool = False, scale: Optional[float] = None,
-                  window=None, dqkv=None, stream=None):
+                  window=None, dqkv=None, stream=None, deterministic: bool = False):
     """Backward of fwd_qkvpacked; the gradient is written packed, [B, N, 3, H, d]."""
     _require(qkv, "qkv")
     if qkv.dim() != 5 or qkv.shape[2] != 3:
@@ -369,7 +372,8 @@ def bwd_qkvpacked(qkv, out, dout, lse, causal: bool = False, scale: Optional[flo
     dqkv = torch.empty_like(qkv) if dqkv is None else dqkv
     _require(dqkv, "dqkv", shape=qkv.shape, device=qkv.device)
     bwd_ex(qkv[:, :, 0], qkv[:, :, 1], qkv[:, :, 2], out, dout, lse, causal=causal, scale=scale,
-           window=window, dq=dqkv[:, :, 0], dk=dqkv[:, :, 1], dv=dqkv[:, :, 2], stream=stream)
+           window=window, dq=dqkv[:, :, 0], dk=dqkv[:, :, 1], dv=dqkv[:, :, 2], stream=stream,
+           deterministic=deterministic)
     return dqkv
 
 

@@ -102,7 +102,7 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* out, floa
                     float scale, void* stream);
 
 /* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator and
- * the per-row D = rowsum(dO * O) vector). Pure function of its arguments. */
+ * the per-row D = rowsum(dO * O) and LSE vectors). Pure function of its arguments. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /*
@@ -117,7 +117,7 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *                        contents on entry are ignored and left undefined.
  * dq is summed over key tiles with fp32 reductions into the workspace in an order
  * that is not fixed, so dq may differ in the last bits between runs; dk and dv are
- * bitwise repeatable.
+ * bitwise repeatable (fa_bwd_ex with deterministic = 1 makes dq repeatable too).
  */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                  const float* lse, void* dq, void* dk, void* dv, int B, int H, int N, int d,
@@ -144,13 +144,19 @@ fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const voi
  * (so dq, dk, dv can be views into one packed [B, N, 3, H, d] gradient). lse is the
  * forward's ([B, H, N] dense, [H, total_tokens] variable length). The workspace is
  * fa_bwd_workspace_size(B, H, N, d) bytes with N the largest sequence length.
- * Errors as fa_bwd and fa_fwd_ex.
+ * deterministic: 0 runs the fused backward of fa_bwd (dq summed over key tiles with
+ * fp32 reductions whose order is not fixed); nonzero runs two kernels instead, one
+ * per key tile writing dk and dv and one per query tile writing dq, each gradient
+ * element written once, so all three gradients are bitwise repeatable on the same
+ * inputs (the flash_attn `deterministic` flag of the MindSpore page, section
+ * 常见问题与解决方案). That path recomputes the scores twice (seven tile products per
+ * tile pair instead of five) and is slower. Errors as fa_bwd and fa_fwd_ex.
  */
 fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out, const void* dout,
                     const float* lse, void* dq, void* dk, void* dv, const int* cu_seqlens,
                     int total_tokens, int B, int H, int N, int d, const long long* row_strides,
-                    int causal, int window_left, int window_right, float scale, void* workspace,
-                    size_t workspace_bytes, void* stream);
+                    int causal, int window_left, int window_right, float scale, int deterministic,
+                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * fa_bwd for callers that cannot allocate device memory. Some callers have no way

@@ -39,7 +39,7 @@ def test_header_and_binding_agree():
 def test_library_exports_every_declared_symbol(lib):
     for name in _header_functions():
         assert hasattr(lib, name), name
-    assert lib.fa_abi_version() == 1
+    assert lib.fa_abi_version() == 2
 
 
 def test_bwd_workspace_size_is_pure_and_padded(lib):
@@ -115,15 +115,16 @@ def test_fwd_ex_argument_errors(lib):
 def test_bwd_ex_argument_errors(lib):
     rs8 = (ctypes.c_longlong * 8)(*([128] * 8))
 
-    def call(rs=rs8, ws=P16, ws_bytes=1 << 30, wr=-1, causal=0):
+    def call(rs=rs8, ws=P16, ws_bytes=1 << 30, wr=-1, causal=0, det=0):
         return lib.fa_bwd_ex(P16, P16, P16, P16, P16, P16, P16, P16, P16, NULL, 0, 1, 2, 128, 64,
-                             rs, causal, -1, wr, 0.125, ws, ws_bytes, NULL)
+                             rs, causal, -1, wr, 0.125, det, ws, ws_bytes, NULL)
 
-    assert call(rs=None) == INVALID
-    bad = (ctypes.c_longlong * 8)(*([128] * 7 + [100]))
-    assert call(rs=bad) == INVALID
-    assert call(causal=1, wr=3) == INVALID
-    assert call(ws=NULL) == WORKSPACE
+    for det in (0, 1):  # the deterministic backward takes the same checks
+        assert call(rs=None, det=det) == INVALID
+        bad = (ctypes.c_longlong * 8)(*([128] * 7 + [100]))
+        assert call(rs=bad, det=det) == INVALID
+        assert call(causal=1, wr=3, det=det) == INVALID
+        assert call(ws=NULL, det=det) == WORKSPACE
 
 
 def test_decode_paged_argument_errors(lib):

@@ -129,7 +129,12 @@ def test_packed_qkv_reaches_the_abi_with_row_strides(lib):
     dqkv = ops.bwd_qkvpacked(qkv, out, out.clone(), lse, causal=True)
     (name, args), = [c for c in lib.calls if c[0] == "fa_bwd_ex"]
     assert list(args[15]) == [3 * H * d] * 3 + [H * d] * 2 + [3 * H * d] * 3
+    assert args[20] == 0  # deterministic off by default
     assert dqkv.shape == qkv.shape
+    lib.calls.clear()
+    ops.bwd_qkvpacked(qkv, out, out.clone(), lse, causal=True, deterministic=True)
+    (name, args), = [c for c in lib.calls if c[0] == "fa_bwd_ex"]
+    assert args[20] == 1
 
 
 def test_packed_qkv_rejects_a_wrong_gradient_buffer(lib):

@@ -34,8 +34,9 @@ class _OracleOps:
         return torch.from_numpy(o).to(q.dtype), torch.from_numpy(l).float()
 
     def bwd_ex(self, q, k, v, out, dout, lse, causal=False, scale=None, window=None,
-               cu_seqlens=None, max_seqlen=None, **kw):
+               cu_seqlens=None, max_seqlen=None, deterministic=False, **kw):
         self.calls.append(("bwd_ex", causal, scale, window, dout.is_contiguous()))
+        self.deterministic = deterministic
         assert dout.is_contiguous()
         wl, wr = (-1, -1) if window is None else window
         args = [self._np(t) for t in (q, k, v, dout)]
@@ -148,14 +149,16 @@ def test_varlen_uses_one_packing(fake):
         interface.flash_attn_varlen_func(q, k, v, cu, cu, 7, 8)
 
 
-def test_dropout_and_deterministic_are_refused(fake):
+def test_dropout_is_refused_and_deterministic_reaches_the_backward(fake):
     q, k, v = _qkv()
     with pytest.raises(NotImplementedError):
         interface.flash_attn_func(q, k, v, dropout_p=0.1)
-    with pytest.raises(NotImplementedError, match="deterministic"):
-        interface.flash_attn_func(q, k, v, deterministic=True)
-    interface.flash_attn_func(q, k, v, deterministic=False)  # the pages' setting
-    assert [c[0] for c in fake.calls] == ["fwd_ex"]
+    for flag in (False, True):  # False is the pages' setting
+        q.grad = None
+        out = interface.flash_attn_func(q, k, v, deterministic=flag)
+        out.sum().backward()
+        assert fake.deterministic is flag
+    assert [c[0] for c in fake.calls] == ["fwd_ex", "bwd_ex", "fwd_ex", "bwd_ex"]
 
 
 def test_kvcache_step_routes_to_decode_and_paged_decode(fake):
