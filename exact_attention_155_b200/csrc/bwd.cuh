@@ -490,20 +490,33 @@ __global__ void __launch_bounds__(448, 1)
       }
       // Local columns c in [qlo_c, qhi_c] are the queries that see this key (window
       // [key - wr, key + wl]); none if the key is past the sequence. Queries past the
-      // sequence have lse2 = +inf, so their P is already 0.
+      // sequence have lse2 = +inf, so their P is already 0. Only tiles where some key of
+      // the warp misses some of the 64 columns (the causal diagonal, window edges, the
+      // sequence end) take the per-element test.
       const int q0 = it * 128 + c0;
       const int qlo_c = !key_ok ? (1 << 30) : (wr < 0 ? -(1 << 30) : key - wr - q0);
       const int qhi_c = wl < 0 ? (1 << 30) : key + wl - q0;
+      const bool edge = __any_sync(0xffffffffu, qlo_c > 0 || qhi_c < 63);
+      const float4* vec4 = reinterpret_cast<const float4*>(vec);  // 16-byte aligned (c0 = 0, 64)
       uint32_t pk[32];
 #pragma unroll
-      for (int c2 = 0; c2 < 32; ++c2) {
-        const int c = 2 * c2;
-        const uint32_t* src = c < 32 ? s0 : s1;
-        const float e0 = ex2_approx(__uint_as_float(src[c & 31]) * sl2 - vec[c]);
-        const float e1 = ex2_approx(__uint_as_float(src[(c + 1) & 31]) * sl2 - vec[c + 1]);
-        const float p0 = (c < qlo_c || c > qhi_c) ? 0.f : e0;
-        const float p1 = (c + 1 < qlo_c || c + 1 > qhi_c) ? 0.f : e1;
-        pk[c2] = pack_bf16x2(p0, p1);
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 lv = vec4[c4];
+        const uint32_t* src = c4 < 8 ? s0 : s1;
+        const int o = (4 * c4) & 31;
+        float e0 = ex2_approx(__uint_as_float(src[o]) * sl2 - lv.x);
+        float e1 = ex2_approx(__uint_as_float(src[o + 1]) * sl2 - lv.y);
+        float e2 = ex2_approx(__uint_as_float(src[o + 2]) * sl2 - lv.z);
+        float e3 = ex2_approx(__uint_as_float(src[o + 3]) * sl2 - lv.w);
+        if (edge) {
+          const int c = 4 * c4;
+          e0 = (c < qlo_c || c > qhi_c) ? 0.f : e0;
+          e1 = (c + 1 < qlo_c || c + 1 > qhi_c) ? 0.f : e1;
+          e2 = (c + 2 < qlo_c || c + 2 > qhi_c) ? 0.f : e2;
+          e3 = (c + 3 < qlo_c || c + 3 > qhi_c) ? 0.f : e3;
+        }
+        pk[2 * c4] = pack_bf16x2(e0, e1);
+        pk[2 * c4 + 1] = pack_bf16x2(e2, e3);
       }
       // P^T of queries [c0, c0 + 64) goes to columns [c0/2, c0/2 + 32): for the second
       // warpgroup those are S^T columns of the first one, which must have loaded them.
@@ -525,7 +538,7 @@ __global__ void __launch_bounds__(448, 1)
         ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDSFree), (n - 1) & 1, abort_flag, kSiteBwdSoftmax));
       if (!ok) break;
       tc_fence_after();
-      const float* dvec = vec + 128;
+      const float4* dvec4 = reinterpret_cast<const float4*>(vec + 128);
       uint32_t dp0[32], dp1[32];
       tmem_ld32(tDP + lane_off + c0, dp0);
       tmem_ld32(tDP + lane_off + c0 + 32, dp1);
@@ -537,13 +550,16 @@ __global__ void __launch_bounds__(448, 1)
         const uint32_t* dp = q == 0 ? dp0 : dp1;
         uint32_t w[16];
 #pragma unroll
-        for (int c2 = 0; c2 < 16; ++c2) {
-          const uint32_t pp = pk[q * 16 + c2];
-          const float p0 = __uint_as_float(pp << 16), p1 = __uint_as_float(pp & 0xFFFF0000u);
-          const int c = q * 32 + 2 * c2;
-          const float d0 = p0 * (__uint_as_float(dp[2 * c2]) - dvec[c]);
-          const float d1 = p1 * (__uint_as_float(dp[2 * c2 + 1]) - dvec[c + 1]);
-          w[c2] = pack_bf16x2(d0, d1);
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 dv = dvec4[q * 8 + c4];
+          const uint32_t pa = pk[q * 16 + 2 * c4], pb = pk[q * 16 + 2 * c4 + 1];
+          float d0, d1, d2, d3;
+          add2(d0, d1, __uint_as_float(dp[4 * c4]), __uint_as_float(dp[4 * c4 + 1]), -dv.x, -dv.y);
+          add2(d2, d3, __uint_as_float(dp[4 * c4 + 2]), __uint_as_float(dp[4 * c4 + 3]), -dv.z, -dv.w);
+          mul2(d0, d1, d0, d1, __uint_as_float(pa << 16), __uint_as_float(pa & 0xFFFF0000u));
+          mul2(d2, d3, d2, d3, __uint_as_float(pb << 16), __uint_as_float(pb & 0xFFFF0000u));
+          w[2 * c4] = pack_bf16x2(d0, d1);
+          w[2 * c4 + 1] = pack_bf16x2(d2, d3);
         }
         // Row r of the dS^T tile, queries c0 + q*32 .. +31 (box `half`), 128-byte swizzle.
         const uint32_t row_base = sDS + half * 16384 + r * 128;
