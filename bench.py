@@ -56,8 +56,8 @@ NOMINAL_HBM_GBS = 8000.0
 # DRAM bytes per launch of the backward main kernel from an ncu capture of the training
 # workload, valid only for the kernel source it was taken on (sha256 of csrc/bwd.cuh);
 # null otherwise.
-BWD_TRAFFIC = {"src_sha256": "00ade1531fe1e214ba9fdbe8ae5ee1f1bf2a53490bebce85486bcab486fb1ad7",
-               "bytes_per_launch": 828.82e6 + 509.35e6}
+BWD_TRAFFIC = {"src_sha256": "d62ee410504e2d96436db9c9a75086c3220e359145f202e3f42a0c79d8bd793a",
+               "bytes_per_launch": 830.88e6 + 511.87e6}
 
 
 def log(*a):
@@ -87,7 +87,8 @@ def src_sha(rel):
 
 # ----------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clock, power and throttle reasons (200 ms period)."""
+    """nvidia-smi sampling of SM clock, power and throttle reasons (50 ms period: the
+    power cap lowers the SM clock for tens of milliseconds at a time under this load)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -103,7 +104,7 @@ class ClockSampler:
         except Exception:
             sel = str(device_index)
         self.cmd = ["nvidia-smi", "-i", sel, f"--query-gpu={self.FIELDS}",
-                    "--format=csv,noheader,nounits", "-lms", "200"]
+                    "--format=csv,noheader,nounits", "-lms", "50"]
 
     def start(self):
         try:
@@ -141,6 +142,7 @@ class ClockSampler:
         reasons = sorted({self.NAMES[i] for r in load for i, f in enumerate(r["flags"])
                           if f.lower() == "active"})
         return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_mhz_min": min(r["sm"] for r in load),
                 "sm_max_mhz": max(r["smax"] for r in rows), "reasons": reasons,
                 "samples": len(load), "power_w_max": pmax}
 
