@@ -7,6 +7,8 @@
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
+#include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <set>
 #include <utility>
@@ -169,14 +171,30 @@ fa_status check_launch(const char* what) {
   return FA_OK;
 }
 
+// Work-unit tickets of the persistent forward: one counter per launch, taken round
+// robin from a small pool in the library's device image and zeroed on the launch's
+// stream right before the kernel (so launches on different streams use different
+// counters unless more than kTicketSlots are in flight at once).
+constexpr int kTicketSlots = 64;
+__device__ unsigned int g_fwd_tickets[kTicketSlots];
+std::atomic<unsigned int> g_ticket_next{0};
+
 template <int D, bool CAUSAL, bool GENERAL>
 fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                     const fa::FwdParams& p, int dev, cudaStream_t stream) {
+                     fa::FwdParams p, int dev, int sms, cudaStream_t stream) {
   using L = fa::FwdLayout<D>;
   auto kern = fa::fwd_kernel<D, CAUSAL, GENERAL>;
   fa_status st = set_smem(kern, L::kAlloc, dev);
   if (st != FA_OK) return st;
-  const unsigned grid = static_cast<unsigned>(p.num_qblocks) * p.B * p.H;
+  void* tickets = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&tickets, g_fwd_tickets);
+  if (e != cudaSuccess) return cuda_fail(e, "fa_fwd: cudaGetSymbolAddress(tickets)");
+  p.ticket = static_cast<unsigned int*>(tickets) + (g_ticket_next.fetch_add(1) % kTicketSlots);
+  if ((e = cudaMemsetAsync(p.ticket, 0, sizeof(unsigned int), stream)) != cudaSuccess)
+    return cuda_fail(e, "fa_fwd: reset the work-unit ticket");
+  // One CTA per SM (the shared memory and TMEM of a CTA fill one), each taking units
+  // until none are left.
+  const unsigned grid = static_cast<unsigned>(std::min(p.num_units, std::max(1, sms)));
   kern<<<grid, L::kThreads, L::kAlloc, stream>>>(mq, mk, mv, p);
   return check_launch("fa_fwd kernel launch");
 }
@@ -307,7 +325,8 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
 
 fa_status run_fwd(const void* q, const void* k, const void* v, void* out, float* lse,
                   const RowLayout& lay, long long rs_q, long long rs_k, long long rs_v,
-                  long long rs_o, int wl, int wr, float scale, int dev, cudaStream_t stream) {
+                  long long rs_o, int wl, int wr, float scale, int dev, int sms,
+                  cudaStream_t stream) {
   CUtensorMap mq, mk, mv;
   fa_status st;
   if ((st = map_rows(&mq, q, lay, rs_q)) != FA_OK) return st;
@@ -318,6 +337,8 @@ fa_status run_fwd(const void* q, const void* k, const void* v, void* out, float*
   p.H = lay.H;
   p.N = lay.N;
   p.num_qblocks = (lay.N + 255) / 256;
+  p.num_units = p.num_qblocks * lay.B * lay.H;  // < 2^31: checked by the callers
+  p.ticket = nullptr;
   // Eight heads: their K and V (8 x 4 MiB at N = 8192) stay in L2 while their CTAs run.
   p.head_group = head_group_for(lay.B * lay.H, 8);
   p.window_left = wl;
@@ -332,13 +353,13 @@ fa_status run_fwd(const void* q, const void* k, const void* v, void* out, float*
   // kernel instance with those tests compiled out.
   const bool general = lay.cu_seqlens != nullptr || wl >= 0 || wr > 0;
   if (lay.d == 64) {
-    if (general) return launch_fwd<64, false, true>(mq, mk, mv, p, dev, stream);
-    return wr == 0 ? launch_fwd<64, true, false>(mq, mk, mv, p, dev, stream)
-                   : launch_fwd<64, false, false>(mq, mk, mv, p, dev, stream);
+    if (general) return launch_fwd<64, false, true>(mq, mk, mv, p, dev, sms, stream);
+    return wr == 0 ? launch_fwd<64, true, false>(mq, mk, mv, p, dev, sms, stream)
+                   : launch_fwd<64, false, false>(mq, mk, mv, p, dev, sms, stream);
   }
-  if (general) return launch_fwd<128, false, true>(mq, mk, mv, p, dev, stream);
-  return wr == 0 ? launch_fwd<128, true, false>(mq, mk, mv, p, dev, stream)
-                 : launch_fwd<128, false, false>(mq, mk, mv, p, dev, stream);
+  if (general) return launch_fwd<128, false, true>(mq, mk, mv, p, dev, sms, stream);
+  return wr == 0 ? launch_fwd<128, true, false>(mq, mk, mv, p, dev, sms, stream)
+                 : launch_fwd<128, false, false>(mq, mk, mv, p, dev, sms, stream);
 }
 
 // Checks shared by the extended entry points; on success fills `lay`, `wr_eff` (the
@@ -456,12 +477,12 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* out, float* 
   const long long nqb = (static_cast<long long>(N) + 255) / 256;
   if (nqb * B * H >= (1LL << 31) || N > (1 << 30) || H > (1 << 20))
     return fail(FA_ERR_INVALID_ARG, "fa_fwd: problem too large (B=%d H=%d N=%d)", B, H, N);
-  int dev = 0;
-  fa_status st = current_device(&dev, nullptr);
+  int dev = 0, sms = 0;
+  fa_status st = current_device(&dev, &sms);
   if (st != FA_OK) return st;
   const RowLayout lay{B, N, H, d, nullptr, 0};
   const long long rs = static_cast<long long>(H) * d;
-  return run_fwd(q, k, v, out, lse, lay, rs, rs, rs, rs, -1, causal ? 0 : -1, scale, dev,
+  return run_fwd(q, k, v, out, lse, lay, rs, rs, rs, rs, -1, causal ? 0 : -1, scale, dev, sms,
                  static_cast<cudaStream_t>(stream));
 }
 
@@ -480,10 +501,10 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* out, floa
   if (!q || !k || !v || !out || !lse) return fail(FA_ERR_INVALID_ARG, "fa_fwd_ex: null pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) || !aligned4(lse))
     return fail(FA_ERR_INVALID_ARG, "fa_fwd_ex: q/k/v/out must be 16-byte aligned, lse 4-byte aligned");
-  int dev = 0;
-  if ((st = current_device(&dev, nullptr)) != FA_OK) return st;
+  int dev = 0, sms = 0;
+  if ((st = current_device(&dev, &sms)) != FA_OK) return st;
   return run_fwd(q, k, v, out, lse, lay, q_row_stride, k_row_stride, v_row_stride, out_row_stride,
-                 window_left, wr, scale, dev, static_cast<cudaStream_t>(stream));
+                 window_left, wr, scale, dev, sms, static_cast<cudaStream_t>(stream));
 }
 
 size_t fa_bwd_workspace_size(int B, int H, int N, int d) {
