@@ -447,15 +447,6 @@ fa_status noalloc_scratch(void** out) {
   return FA_OK;
 }
 
-__global__ void exp2_poly_kernel(const float* x, float* y, int n) {
-  const int i = (blockIdx.x * blockDim.x + threadIdx.x) * 2;
-  if (i >= n) return;
-  float a = x[i], b = (i + 1 < n) ? x[i + 1] : 0.f;
-  fa::exp2_poly2(a, b);
-  y[i] = a;
-  if (i + 1 < n) y[i + 1] = b;
-}
-
 }  // namespace
 
 // =============================================================================
@@ -800,17 +791,6 @@ fa_status fa_debug_timeout_probe(long long limit_cycles, void* stream) {
   if (st != FA_OK) return st;
   timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_cycles);
   return check_launch("fa_debug_timeout_probe launch");
-}
-
-fa_status fa_debug_exp2(const float* x, float* y, int n, void* stream) {
-  if (n < 0) return fail(FA_ERR_INVALID_ARG, "fa_debug_exp2: n < 0");
-  if (n == 0) return FA_OK;
-  if (!x || !y) return fail(FA_ERR_INVALID_ARG, "fa_debug_exp2: null pointer");
-  fa_status st = current_device(nullptr, nullptr);
-  if (st != FA_OK) return st;
-  const int pairs = (n + 1) / 2;
-  exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  return check_launch("fa_debug_exp2 launch");
 }
 
 }  // extern "C"

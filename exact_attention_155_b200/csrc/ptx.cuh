@@ -302,17 +302,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// The same packing on the integer pipe (no conversion unit): round to nearest with
-// ties away from zero by adding half a bf16 ulp to the fp32 bit pattern (a carry
-// into the exponent is the correct rounding), then keep the two high halves with one
-// byte permute. Differs from round-to-nearest-even only on exact ties. For finite
-// inputs below the bf16 overflow threshold, which is all the softmax produces.
-__device__ __forceinline__ uint32_t pack_bf16x2_alu(float lo, float hi) {
-  const uint32_t a = __float_as_uint(lo) + 0x8000u;
-  const uint32_t b = __float_as_uint(hi) + 0x8000u;
-  return __byte_perm(a, b, 0x7632);  // bytes 2,3 of a, then bytes 2,3 of b
-}
-
 // Packed fp32x2 arithmetic (sm_100): two lanes of work per instruction.
 __device__ __forceinline__ void fma2(float& d0, float& d1, float a0, float a1, float b0, float b1,
                                      float c0, float c1) {
@@ -347,35 +336,6 @@ __device__ __forceinline__ float min3f(float a, float b, float c) {
   asm("min.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
-// 2^x for two values without the MUFU unit (FMA and integer pipes only), used for a
-// fraction of the softmax exponentials so both pipes share the work. Method: j =
-// round(x) by adding and subtracting 1.5 * 2^23, f = x - j in [-1/2, 1/2], 2^f by a
-// cubic fitted by least squares on Chebyshev nodes (coefficients from
-// csrc/gen_exp2_poly.py, max relative error 1.14e-4), and j added to the exponent
-// field. x is clamped to >= -126, where the result (about 1e-38) is negligible
-// next to a softmax row sum of at least 1.
-__device__ __forceinline__ void exp2_poly2(float& a, float& b) {
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c1 = 6.933686137e-01f, c2 = 2.422178388e-01f, c3 = 5.459282547e-02f;
-  a = fmaxf(a, -126.f);
-  b = fmaxf(b, -126.f);
-  float ta, tb, ja, jb, fa, fb, pa, pb;
-  add2(ta, tb, a, b, kMagic, kMagic);
-  add2(ja, jb, ta, tb, -kMagic, -kMagic);
-  fma2(fa, fb, ja, jb, -1.f, -1.f, a, b);
-  fma2(pa, pb, fa, fb, c3, c3, c2, c2);
-  fma2(pa, pb, pa, pb, fa, fb, c1, c1);
-  fma2(pa, pb, pa, pb, fa, fb, 1.f, 1.f);
-  // The low mantissa bits of t hold j + 2^22; shifted into the exponent field the
-  // 2^22 term leaves the 32-bit word, so (bits(t) << 23) adds exactly j to the exponent.
-  a = __uint_as_float(__float_as_uint(pa) + (__float_as_uint(ta) << 23));
-  b = __uint_as_float(__float_as_uint(pb) + (__float_as_uint(tb) << 23));
-}
-
-__device__ __forceinline__ void red_add_f32(float* addr, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(v) : "memory");
-}
-
 // Named barriers (ids 1..15; 0 is __syncthreads).
 // Barrier over `nthreads` threads that also returns the OR of every thread's predicate.
 __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {

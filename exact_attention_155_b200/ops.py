@@ -68,7 +68,6 @@ _SIGNATURES = {
     "fa_device_status": (_c_int, [_c_void_p, ctypes.POINTER(ctypes.c_uint),
                                   ctypes.POINTER(ctypes.c_uint)]),
     "fa_debug_timeout_probe": (_c_int, [ctypes.c_longlong, _c_void_p]),
-    "fa_debug_exp2": (_c_int, [_c_void_p, _c_void_p, _c_int, _c_void_p]),
     "fa_abi_version": (_c_int, []),
 }
 
@@ -498,14 +497,6 @@ def device_status(stream=None):
     site, info = ctypes.c_uint(0), ctypes.c_uint(0)
     st = lib.fa_device_status(_stream(stream), ctypes.byref(site), ctypes.byref(info))
     return st, site.value, info.value
-
-
-def debug_exp2(x: torch.Tensor, stream=None) -> torch.Tensor:
-    """2^x by the kernels' FMA-pipe polynomial (fp32 CUDA tensor in, same shape out)."""
-    _require(x, "x", torch.float32)
-    y = torch.empty_like(x)
-    _check(load_library().fa_debug_exp2(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
-    return y
 
 
 def debug_timeout_probe(limit_cycles: int, stream=None):

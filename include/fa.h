@@ -293,13 +293,6 @@ fa_status fa_device_status(void* stream, unsigned int* site_out, unsigned int* i
  */
 fa_status fa_debug_timeout_probe(long long limit_cycles, void* stream);
 
-/*
- * Diagnostic: y[i] = 2^x[i] computed by the kernels' FMA-pipe polynomial (the one
- * that takes a share of the softmax exponentials instead of the MUFU unit), for
- * n device floats, so tests can bound its error against an exact exp2.
- */
-fa_status fa_debug_exp2(const float* x, float* y, int n, void* stream);
-
 /* Library ABI version (incremented on any signature change). */
 int fa_abi_version(void);
 
