@@ -97,3 +97,22 @@ def test_emulated_ring_bwd_matches_whole_sequence(world, causal, d):
     grads = ring_attention_bwd_emulated(q, k, v, out, do, lse, world, causal=causal, scale=sc)
     torch.cuda.synchronize()
     check_grads(grads, inp, causal, sc)
+
+
+@pytest.mark.parametrize("world", [1, 2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_emulated_zigzag_ring_matches_whole_sequence(world, causal, d):
+    """The zigzag layout (rank r holds chunks r and 2R-1-r) for 1, 2 and 4 shards, the
+    exchange emulated in one process: forward output and LSE, and the gradients, against
+    the oracle over the whole sequence (given and returned in sequence order)."""
+    B, N, H = 2, 1024, 2
+    inp = make_inputs(B, N, H, d, 9995 + world + d + int(causal))
+    q, k, v, do = (inp[n].cuda() for n in ("q", "k", "v", "dout"))
+    sc = default_scale(d)
+    out, lse = ring_attention_fwd_emulated(q, k, v, world, causal=causal, scale=sc, layout="zigzag")
+    grads = ring_attention_bwd_emulated(q, k, v, out, do, lse, world, causal=causal, scale=sc,
+                                        layout="zigzag")
+    torch.cuda.synchronize()
+    check_fwd(out, lse, inp, causal, sc)
+    check_grads(grads, inp, causal, sc)

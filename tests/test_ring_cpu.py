@@ -464,3 +464,118 @@ def test_ring_flash_attn_func_autograd_over_gloo():
         np.testing.assert_allclose(o, ref_o[:, rows], atol=_ATOL)
         for g, r in zip(grads, refs):
             np.testing.assert_allclose(g, r[:, rows], atol=_ATOL)
+
+
+# ----------------------------------------------------------------- zigzag layout
+@pytest.mark.parametrize("world", [1, 2, 3, 4, 5])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zigzag_plan_covers_every_visible_chunk_pair_once_with_equal_work(world, causal):
+    """Brute force over the 2R chunks: the plans of all (rank, step) name each chunk
+    pair a query chunk sees exactly once (causal on its own chunk), and every rank does
+    the same work at every step (a causal chunk pair counts half)."""
+    from exact_attention_155_b200.ring import zigzag_plan
+    chunk = lambda r, half: r if half == 0 else 2 * world - 1 - r
+    seen = {}
+    for rank in range(world):
+        for s, src, _ in ring_schedule(rank, world, False):
+            work = 0.0
+            for a, b, mode in zigzag_plan(rank, src, causal):
+                qc, kc = chunk(rank, a), chunk(src, b)
+                assert (qc, kc) not in seen
+                seen[(qc, kc)] = mode
+                work += 0.5 if mode == CAUSAL else 1.0
+            assert work == (2.0 if causal else 4.0)
+    want = {(qc, kc): (CAUSAL if qc == kc else FULL) for qc in range(2 * world)
+            for kc in range(2 * world) if not causal or kc <= qc}
+    if not causal:
+        want = {key: FULL for key in want}
+    assert seen == want
+
+
+@pytest.mark.parametrize("world", [1, 2, 3])
+def test_zigzag_shard_and_unshard_round_trip(world):
+    from exact_attention_155_b200.ring import zigzag_shard, zigzag_unshard
+    x = torch.arange(2 * 4 * world * 3, dtype=torch.float32).reshape(2, 4 * world, 3)
+    shards = [zigzag_shard(x, r, world) for r in range(world)]
+    c = 2
+    assert torch.equal(shards[0][:, :c], x[:, :c])                      # chunk 0
+    assert torch.equal(shards[0][:, c:], x[:, (2 * world - 1) * c:])     # chunk 2R-1
+    assert torch.equal(zigzag_unshard(shards), x)
+    with pytest.raises(ValueError):
+        zigzag_shard(x[:, :3], 0, world + 1)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_emulated_zigzag_ring_fwd_and_bwd_on_cpu(world, causal, monkeypatch):
+    """The zigzag emulation's bookkeeping (chunk halves, per-chunk sums, reassembly in
+    sequence order) with the oracle standing in for the kernels."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_155_b200 import ring
+    monkeypatch.setattr(ring, "_attend_and_merge", _oracle_attend_and_merge)
+    monkeypatch.setattr(ring, "_pair_terms", _oracle_pair_terms)
+    monkeypatch.setattr(ring, "_add_terms", _oracle_add_terms)
+    monkeypatch.setattr(ring, "_to_bf16", _oracle_to_bf16)
+    full = _full_inputs(world, S=8, seed=199 + world)
+    q, k, v, do = full
+    out, lse = ring.ring_attention_fwd_emulated(q, k, v, world, causal=causal, scale=0.7,
+                                                layout=ring.ZIGZAG)
+    ref_o, ref_l = oracle.attention_forward(*[t.numpy() for t in full[:3]], causal=causal, scale=0.7)
+    np.testing.assert_allclose(out.numpy(), ref_o, atol=_ATOL)
+    np.testing.assert_allclose(lse.numpy(), ref_l, atol=_ATOL)
+    grads = ring.ring_attention_bwd_emulated(q, k, v, out, do, lse, world, causal=causal, scale=0.7,
+                                             layout=ring.ZIGZAG)
+    refs = oracle.attention_backward(*[t.numpy() for t in full], causal=causal, scale=0.7)
+    for g, r in zip(grads, refs):
+        np.testing.assert_allclose(g.numpy(), r, atol=_ATOL)
+
+
+def _zigzag_worker(rank, world, port, causal, q):
+    """ring_attention_fwd and ring_attention_bwd in the zigzag layout over gloo with the
+    oracle standing in for the kernels; returns this rank's shards of the results."""
+    import oracle
+    from exact_attention_155_b200 import ring
+
+    _use_oracle_seams(ring)
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        full = _full_inputs(world, S=8, seed=4242 + world)
+        zz = lambda t, dim=1: ring.zigzag_shard(t, rank, world, dim)
+        qs, ks, vs, dos = (zz(t).contiguous() for t in full)
+        out, lse = ring.ring_attention_fwd(qs, ks, vs, causal=causal, scale=0.5, layout=ring.ZIGZAG)
+        # The backward from the oracle's whole-sequence forward, as the ring forward gives it.
+        ro, rl = oracle.attention_forward(*[t.numpy() for t in full[:3]], causal=causal, scale=0.5)
+        os_ = zz(torch.from_numpy(ro)).contiguous()
+        ls = zz(torch.from_numpy(rl), 2).contiguous()
+        grads = ring.ring_attention_bwd(qs, ks, vs, os_, dos, ls, causal=causal, scale=0.5,
+                                        layout=ring.ZIGZAG)
+        q.put((rank, out.numpy(), lse.numpy(), [g.numpy() for g in grads], [t.numpy() for t in full]))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("causal", [False, True])
+def test_zigzag_ring_driver_over_gloo(world, causal):
+    """Each rank's zigzag shards of the output, LSE and gradients equal the oracle's over
+    the whole sequence."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_155_b200.ring import zigzag_shard
+    got = _spawn(_zigzag_worker, world, causal)
+    full = [torch.from_numpy(t) for t in got[0][3]]
+    ref_o, ref_l = oracle.attention_forward(*[t.numpy() for t in full[:3]], causal=causal, scale=0.5)
+    refs = oracle.attention_backward(*[t.numpy() for t in full], causal=causal, scale=0.5)
+    zz = lambda a, r, dim=1: zigzag_shard(torch.from_numpy(a), r, world, dim).numpy()
+    for rank in range(world):
+        o, l, grads, _ = got[rank]
+        np.testing.assert_allclose(o, zz(ref_o, rank), atol=_ATOL)
+        np.testing.assert_allclose(l, zz(ref_l, rank, 2), atol=_ATOL)
+        for g, r in zip(grads, refs):
+            np.testing.assert_allclose(g, zz(r, rank), atol=_ATOL)
