@@ -593,6 +593,33 @@ def run_ours(args, rank, world, local_rank):
         for _ in range(2):
             ring_fn()
         rms = timed_events(torch, ring_fn, 5)
+
+        def ring_parallel_ms(xq, xk, xv, layout):
+            """Time of a parallel run of the emulated ranks: per step, the slowest rank's
+            kernels (CUDA events around each rank's work at each step), summed over steps;
+            the exchange (NCCL point-to-point, overlapped with the compute) is not in it."""
+            ring_attention_fwd_emulated(xq, xk, xv, 4, causal=True, scale=scale, layout=layout)
+            best = None
+            for _ in range(3):
+                evs = []
+                ring_attention_fwd_emulated(xq, xk, xv, 4, causal=True, scale=scale, layout=layout,
+                                            step_events=evs)
+                torch.cuda.synchronize()
+                per_step = {}
+                for _r, st, a, b in evs:
+                    per_step.setdefault(st, []).append(a.elapsed_time(b))
+                ms = sum(max(v) for v in per_step.values())
+                best = ms if best is None else min(best, ms)
+            return best
+        ring_par = {p["N"]: {lay: ring_parallel_ms(rq, rk, rv, lay) for lay in ("contiguous", "zigzag")}}
+        del rq, rk, rv
+        # The same estimate on a 32768-token sequence (8192 rows per rank), the length where
+        # splitting the sequence over GPUs is the point.
+        RN = 32768
+        rin = attention_inputs(1, RN, p["H"], p["d"], seed=1009, with_dout=False)
+        rq, rk, rv = (rin[n].to(dev) for n in ("q", "k", "v"))
+        del rin
+        ring_par[RN] = {lay: ring_parallel_ms(rq, rk, rv, lay) for lay in ("contiguous", "zigzag")}
         del rq, rk, rv
         parts = {
             "prefill_fwd": {"workload": "causal fwd B=1 H=32 N=8192 d=128", "value": ptf,
@@ -631,7 +658,15 @@ def run_ours(args, rank, world, local_rank):
                             "(ring schedule, partial attention + LSE merge per shard pair)",
                 "value": fwd_flops(p["B"], p["H"], p["N"], p["d"], True) / (rms * 1e-3) / 1e12,
                 "unit": "TFLOP/s", "ms": rms,
-                "note": "exchange is indexing here; NCCL send/recv only with several GPUs"},
+                "parallel_estimate": {
+                    f"N={n}": {lay: {"ms": ms, "tflops_per_gpu":
+                                     fwd_flops(1, p["H"], n, p["d"], True) / 4 / (ms * 1e-3) / 1e12}
+                               for lay, ms in v.items()}
+                    for n, v in ring_par.items()},
+                "note": "value: all 4 ranks run one after another on this GPU (exchange is "
+                        "indexing); parallel_estimate: sum over the 4 steps of the slowest "
+                        "rank's kernel time, contiguous shards vs zigzag chunks, at N = 8192 "
+                        "and N = 32768"},
             "window_causal": {
                 "workload": f"causal sliding window {wwin[0]}, B=1 H=32 N=16384 d=128",
                 "fwd_tflops": wf_fl / (wf_ms * 1e-3) / 1e12, "fwd_ms": wf_ms,
