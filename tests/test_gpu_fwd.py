@@ -79,3 +79,27 @@ def test_fwd_rejects_bad_inputs():
     with pytest.raises(fa.FAError, match="UNSUPPORTED"):
         z = torch.zeros(1, 128, 2, 96, dtype=torch.bfloat16, device="cuda")
         fa.fwd(z, z, z)
+
+
+def test_fwd_on_concurrent_streams_matches_one_stream():
+    """The persistent forward takes work units from a per-launch ticket counter; calls
+    in flight on different streams use different counters, so overlapping launches
+    (many of them, wrapping the counter pool) give the same bits as one at a time."""
+    shapes = [(1, 2048, 8, 128, True), (2, 777, 4, 64, False), (1, 4096, 4, 128, True)]
+    inputs = [make_inputs(B, N, H, d, 7400 + i, with_dout=False) for i, (B, N, H, d, _) in enumerate(shapes)]
+    dev = [tuple(inp[n].cuda() for n in ("q", "k", "v")) for inp in inputs]
+    ref = []
+    for (q, k, v), (_, _, _, d, causal) in zip(dev, shapes):
+        ref.append(fa.fwd(q, k, v, causal=causal, scale=default_scale(d)))
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream() for _ in shapes]
+    outs = [[None] * 30 for _ in shapes]
+    for rep in range(30):  # 90 launches: more than the pool of counters
+        for i, ((q, k, v), (_, _, _, d, causal), s) in enumerate(zip(dev, shapes, streams)):
+            with torch.cuda.stream(s):
+                outs[i][rep] = fa.fwd(q, k, v, causal=causal, scale=default_scale(d))
+    torch.cuda.synchronize()
+    assert fa.device_status()[0] == 0
+    for i in range(len(shapes)):
+        for o, l in outs[i]:
+            assert torch.equal(o, ref[i][0]) and torch.equal(l, ref[i][1])
