@@ -123,15 +123,20 @@ __global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
   // Element offset of cache row r from this (b, h)'s row 0 (contiguous) or from the
   // cache base (paged), or -1 for a page id outside [0, num_pages), which is reported
   // and never dereferenced.
-  auto row_off = [&](int r) -> long long {
-    if (!PAGED) return static_cast<long long>(r) * static_cast<long long>(row_stride);
-    const int pg = __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + (r >> p.page_shift));
+  auto table_at = [&](int r) -> int {
+    return __ldg(p.block_table + static_cast<size_t>(b) * p.max_blocks + (r >> p.page_shift));
+  };
+  auto paged_off = [&](int pg, int r) -> long long {
     if (pg < 0 || pg >= p.num_pages) {
       report(kDevBadInput, kSiteDecodePage, b);
       return -1;
     }
     return ((static_cast<long long>(pg) << p.page_shift) + (r & ((1 << p.page_shift) - 1))) *
            static_cast<long long>(row_stride);
+  };
+  auto row_off = [&](int r) -> long long {
+    if (!PAGED) return static_cast<long long>(r) * static_cast<long long>(row_stride);
+    return paged_off(table_at(r), r);
   };
   const uint16_t* kn = append ? p.k_new + bh * D + sub * 8 : nullptr;
   const uint16_t* vn = append ? p.v_new + bh * D + sub * 8 : nullptr;
@@ -161,8 +166,24 @@ __global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) o[i] = 0.f;
 
+  // Paged: the page ids of the next row step are read while this step's K/V loads are
+  // in flight, so no K/V load waits on a block-table read.
+  auto page_id = [&](int r) -> int { return r < k1 ? table_at(r) : 0; };
+  int pg_next[U];
+  if (PAGED) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) pg_next[u] = page_id(k0 + warp * RPW + u * RSTEP + grp);
+  }
   // Rows handled by this lane group: k0 + warp*RPW + grp + RSTEP*t, t = 0, 1, ...
   for (int base = k0 + warp * RPW; base < k1; base += U * RSTEP) {
+    int pg[U];
+    if (PAGED) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        pg[u] = pg_next[u];
+        pg_next[u] = page_id(base + U * RSTEP + u * RSTEP + grp);
+      }
+    }
     uint4 kv[U], vv[U];
     bool live[U];  // row inside the chunk with a readable source
 #pragma unroll
@@ -173,7 +194,7 @@ __global__ void __launch_bounds__(128) decode_kernel(const DecodeParams p) {
       live[u] = false;
       if (kb < k1) {
         const bool is_new = do_append && kb == L;
-        const long long off = is_new ? 0 : row_off(kb);
+        const long long off = is_new ? 0 : PAGED ? paged_off(pg[u], kb) : row_off(kb);
         if (is_new || off >= 0) {
           live[u] = true;
           kv[u] = __ldg(reinterpret_cast<const uint4*>(is_new ? kn : kc + off));

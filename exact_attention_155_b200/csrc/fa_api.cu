@@ -202,12 +202,15 @@ fa_status launch_fwd(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 
 template <int D, bool CAUSAL, bool GENERAL>
 fa_status launch_bwd_main(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                          const CUtensorMap& mdo, const fa::BwdParams& p, int dev, cudaStream_t stream) {
+                          const CUtensorMap& mdo, const fa::BwdParams& p, int dev, int sms,
+                          cudaStream_t stream) {
   using L = fa::BwdLayout<D>;
   auto kern = fa::bwd_kernel<D, CAUSAL, GENERAL>;
   fa_status st = set_smem(kern, L::kBytes, dev);
   if (st != FA_OK) return st;
-  const unsigned grid = static_cast<unsigned>(p.nqt) * p.B * p.H;
+  // Persistent: one CTA per SM (its shared memory and TMEM fill one), each taking
+  // units from the workspace counter until none are left.
+  const unsigned grid = static_cast<unsigned>(std::min(p.num_units, std::max(1, sms)));
   kern<<<grid, L::kThreads, L::kBytes, stream>>>(mq, mk, mv, mdo, p);
   return check_launch("fa_bwd main kernel launch");
 }
@@ -242,7 +245,7 @@ struct BwdStrides {
 fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,
                   const float* lse, void* dq, void* dk, void* dv, const RowLayout& lay,
                   const BwdStrides& rs, int wl, int wr, float scale, void* workspace,
-                  const fa::BwdWorkspace& ws, bool deterministic, int dev, cudaStream_t stream,
+                  const fa::BwdWorkspace& ws, bool deterministic, int dev, int sms, cudaStream_t stream,
                   cudaEvent_t ev_start, cudaEvent_t ev_stop) {
   const int B = lay.B, H = lay.H, N = lay.N, d = lay.d;
   CUtensorMap mq, mk, mv, mdo;
@@ -276,6 +279,8 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
   char* w = static_cast<char*>(workspace);
   // The deterministic kernels write dq directly: no fp32 accumulator to zero or convert.
   p.dq_acc = deterministic ? nullptr : reinterpret_cast<float*>(w + ws.dq_off);
+  p.num_units = p.nqt * B * H;  // < 2^31: checked by the callers
+  p.ticket = deterministic ? nullptr : reinterpret_cast<unsigned int*>(w + ws.ticket_off);
   p.lse2 = reinterpret_cast<float*>(w + ws.lse2_off);
   p.dvec = reinterpret_cast<float*>(w + ws.dvec_off);
   p.dq = static_cast<uint16_t*>(dq);
@@ -306,13 +311,13 @@ fa_status run_bwd(const void* q, const void* k, const void* v, const void* out, 
     return FA_OK;
   }
   if (d == 64)
-    st = general ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, dev, stream)
-         : wr == 0 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, dev, stream)
-                   : launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, dev, stream);
+    st = general ? launch_bwd_main<64, false, true>(mq, mk, mv, mdo, p, dev, sms, stream)
+         : wr == 0 ? launch_bwd_main<64, true, false>(mq, mk, mv, mdo, p, dev, sms, stream)
+                   : launch_bwd_main<64, false, false>(mq, mk, mv, mdo, p, dev, sms, stream);
   else
-    st = general ? launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, dev, stream)
-         : wr == 0 ? launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, dev, stream)
-                   : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, dev, stream);
+    st = general ? launch_bwd_main<128, false, true>(mq, mk, mv, mdo, p, dev, sms, stream)
+         : wr == 0 ? launch_bwd_main<128, true, false>(mq, mk, mv, mdo, p, dev, sms, stream)
+                   : launch_bwd_main<128, false, false>(mq, mk, mv, mdo, p, dev, sms, stream);
   if (st != FA_OK) return st;
   if (ev_stop && (e = cudaEventRecord(ev_stop, stream)) != cudaSuccess)
     return cuda_fail(e, "fa_bwd_profiled: record stop event");
@@ -525,14 +530,14 @@ fa_status fa_bwd_profiled(const void* q, const void* k, const void* v, const voi
     return fail(FA_ERR_WORKSPACE, "fa_bwd: workspace needs %zu bytes, got %zu", ws.total, workspace_bytes);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(FA_ERR_INVALID_ARG, "fa_bwd: workspace must be 256-byte aligned");
-  int dev = 0;
-  fa_status st = current_device(&dev, nullptr);
+  int dev = 0, sms = 0;
+  fa_status st = current_device(&dev, &sms);
   if (st != FA_OK) return st;
   const RowLayout lay{B, N, H, d, nullptr, 0};
   const long long rs = static_cast<long long>(H) * d;
   const BwdStrides strides{rs, rs, rs, rs, rs, rs, rs, rs};
   return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, lay, strides, -1, causal ? 0 : -1, scale,
-                 workspace, ws, false, dev, static_cast<cudaStream_t>(stream),
+                 workspace, ws, false, dev, sms, static_cast<cudaStream_t>(stream),
                  static_cast<cudaEvent_t>(main_start), static_cast<cudaEvent_t>(main_stop));
 }
 
@@ -558,12 +563,12 @@ fa_status fa_bwd_ex(const void* q, const void* k, const void* v, const void* out
     return fail(FA_ERR_WORKSPACE, "fa_bwd_ex: workspace needs %zu bytes, got %zu", ws.total, workspace_bytes);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(FA_ERR_INVALID_ARG, "fa_bwd_ex: workspace must be 256-byte aligned");
-  int dev = 0;
-  if ((st = current_device(&dev, nullptr)) != FA_OK) return st;
+  int dev = 0, sms = 0;
+  if ((st = current_device(&dev, &sms)) != FA_OK) return st;
   const BwdStrides strides{row_strides[0], row_strides[1], row_strides[2], row_strides[3],
                            row_strides[4], row_strides[5], row_strides[6], row_strides[7]};
   return run_bwd(q, k, v, out, dout, lse, dq, dk, dv, lay, strides, window_left, wr, scale, workspace,
-                 ws, deterministic != 0, dev, static_cast<cudaStream_t>(stream), nullptr, nullptr);
+                 ws, deterministic != 0, dev, sms, static_cast<cudaStream_t>(stream), nullptr, nullptr);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* out, const void* dout,

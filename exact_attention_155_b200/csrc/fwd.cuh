@@ -450,7 +450,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     bool ok = true;
     for (int k = 0; ok; ++k) {
       int u = -1;
-      if (!(ok = next_unit(k, &u)) || u < 0) break;
+      // The warps of a lane quarter share named barriers, so they take the same
+      // decision even if an abort lands while some of them are still waiting.
+      ok = named_bar_and(kBarVote, NTQ, next_unit(k, &u));
+      if (!ok || u < 0) break;
       const FwdUnit w = fwd_unit<CAUSAL, GENERAL>(p, u, false);
       if (w.nkv_max == 0) continue;
       const int seqlen = w.seqlen;

@@ -101,8 +101,9 @@ fa_status fa_fwd_ex(const void* q, const void* k, const void* v, void* out, floa
                     long long out_row_stride, int causal, int window_left, int window_right,
                     float scale, void* stream);
 
-/* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator and
- * the per-row D = rowsum(dO * O) and LSE vectors). Pure function of its arguments. */
+/* Bytes of device workspace fa_bwd needs for these sizes (fp32 dQ accumulator, the
+ * per-row D = rowsum(dO * O) and LSE vectors, and the work-unit counter of the
+ * persistent kernel). Pure function of its arguments. */
 size_t fa_bwd_workspace_size(int B, int H, int N, int d);
 
 /*

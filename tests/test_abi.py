@@ -43,12 +43,13 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_bwd_workspace_size_is_pure_and_padded(lib):
-    # dQ accumulator [B,H,Np,d] fp32 + two [B,H,Np] fp32 vectors, Np = roundup(N, 128).
+    # dQ accumulator [B,H,Np,d] fp32 + two [B,H,Np] fp32 vectors, Np = roundup(N, 128),
+    # + 256 bytes for the work-unit counter of the persistent kernel.
     for (B, H, N, d) in [(1, 2, 128, 64), (2, 3, 129, 128), (1, 32, 16384, 128)]:
         Np = (N + 127) // 128 * 128
         rows = B * H * Np
         r256 = lambda x: (x + 255) // 256 * 256
-        expect = r256(rows * d * 4) + 2 * r256(rows * 4)
+        expect = r256(rows * d * 4) + 2 * r256(rows * 4) + 256
         assert lib.fa_bwd_workspace_size(B, H, N, d) == expect
     assert lib.fa_bwd_workspace_size(1, 1, 128, 96) == 0
     assert lib.fa_bwd_workspace_size(0, 1, 128, 64) == 0
