@@ -56,8 +56,8 @@ NOMINAL_HBM_GBS = 8000.0
 # DRAM bytes per launch of the backward main kernel from an ncu capture of the training
 # workload, valid only for the kernel source it was taken on (sha256 of csrc/bwd.cuh);
 # null otherwise.
-BWD_TRAFFIC = {"src_sha256": "d62ee410504e2d96436db9c9a75086c3220e359145f202e3f42a0c79d8bd793a",
-               "bytes_per_launch": 830.88e6 + 511.87e6}
+BWD_TRAFFIC = {"src_sha256": "a6cb1fd351a648cbda1030aa8c9b7cceefe1ece7e963747d67977643a5a8d993",
+               "bytes_per_launch": 830.83e6 + 511.41e6}
 
 
 def log(*a):

@@ -88,6 +88,37 @@ def test_varlen_forward_and_backward(d, causal, lens):
     _cmp_grads(grads, refs)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_varlen_many_short_sequences(d, causal):
+    """60 sequences of 0-300 tokens and one of 1000: thousands of work units, most of
+    them past the end of their (short or empty) sequence, spread over more units than
+    SMs, so the persistent kernels skip units and take several each."""
+    g = torch.Generator().manual_seed(9400 + d + int(causal))
+    lens = [int(x) for x in torch.randint(0, 301, (60,), generator=g)]
+    lens[7] = 0
+    lens[33] = 0
+    lens[20] = 1000
+    H = 4
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    total = int(cu[-1])
+    q, k, v, do = (bf16_randn((total, H, d), g) for _ in range(4))
+    sc = default_scale(d)
+    cu_t = torch.from_numpy(cu).cuda()
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, do))
+    out, lse = fa.fwd_ex(qc, kc, vc, causal=causal, scale=sc, cu_seqlens=cu_t, max_seqlen=max(lens))
+    grads = fa.bwd_ex(qc, kc, vc, out, doc, lse, causal=causal, scale=sc, cu_seqlens=cu_t,
+                      max_seqlen=max(lens))
+    torch.cuda.synchronize()
+    assert fa.device_status()[0] == 0
+    ref_o, ref_l = oracle.attention_forward_varlen(to_f64(q), to_f64(k), to_f64(v), cu,
+                                                   causal=causal, scale=sc)
+    _cmp_out(out, lse, ref_o, ref_l)
+    refs = oracle.attention_backward_varlen(to_f64(q), to_f64(k), to_f64(v), to_f64(do), cu,
+                                            causal=causal, scale=sc)
+    _cmp_grads(grads, refs)
+
+
 WINDOW_CASES = [(True, 64, 0), (True, 300, 0), (True, 0, 0), (False, 100, 50), (False, -1, 37),
                 (False, 200, -1), (False, 129, 129)]
 
