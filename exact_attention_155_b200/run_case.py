@@ -6,6 +6,7 @@ kernels for the chosen op, on seeded N(0,1) bf16 inputs.
   python -m exact_attention_155_b200.run_case --op fwd --B 1 --H 32 --N 8192 --d 128 --causal 1
   python -m exact_attention_155_b200.run_case --op bwd --N 8192
   python -m exact_attention_155_b200.run_case --op decode --B 32 --H 16 --d 64 --N 2048
+  python -m exact_attention_155_b200.run_case --op decode --B 32 --H 16 --d 64 --N 2048 --page-size 64
 """
 from __future__ import annotations
 
@@ -28,6 +29,8 @@ def main(argv=None):
     ap.add_argument("--d", type=int, default=128)
     ap.add_argument("--causal", type=int, default=1)
     ap.add_argument("--reps", type=int, default=2)
+    ap.add_argument("--page-size", type=int, default=0,
+                    help="decode: >0 runs the paged cache (pages of this many rows at shuffled pool positions)")
     a = ap.parse_args(argv)
 
     import torch
@@ -54,8 +57,22 @@ def main(argv=None):
         kc, vc, qs, _, _ = decode_inputs(a.B, a.H, a.d, a.N, 1, seed=4243)
         kc, vc, q = kc.to(dev), vc.to(dev), qs[0].to(dev)
         seq = torch.full((a.B,), a.N, dtype=torch.int32, device=dev)
-        for _ in range(a.reps):
-            fa.decode(q, kc, vc, seq, scale=scale)
+        if a.page_size > 0:
+            if a.N % a.page_size:
+                raise SystemExit("--N must be a multiple of --page-size")
+            nb = a.N // a.page_size
+            perm = torch.randperm(a.B * nb, generator=torch.Generator().manual_seed(1008)).to(dev)
+            table = perm.view(a.B, nb).to(torch.int32)
+            shape = (a.B * nb, a.page_size, a.H, a.d)
+            kp = torch.empty(shape, dtype=torch.bfloat16, device=dev)
+            vp = torch.empty_like(kp)
+            kp[perm] = kc.view(shape)
+            vp[perm] = vc.view(shape)
+            for _ in range(a.reps):
+                fa.decode_paged(q, kp, vp, table, seq, scale=scale)
+        else:
+            for _ in range(a.reps):
+                fa.decode(q, kc, vc, seq, scale=scale)
     torch.cuda.synchronize()
     st = fa.device_status()
     if st[0] != 0:
