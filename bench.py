@@ -56,8 +56,8 @@ NOMINAL_HBM_GBS = 8000.0
 # DRAM bytes per launch of the backward main kernel from an ncu capture of the training
 # workload, valid only for the kernel source it was taken on (sha256 of csrc/bwd.cuh);
 # null otherwise.
-BWD_TRAFFIC = {"src_sha256": "a6cb1fd351a648cbda1030aa8c9b7cceefe1ece7e963747d67977643a5a8d993",
-               "bytes_per_launch": 830.83e6 + 511.41e6}
+BWD_TRAFFIC = {"src_sha256": "9ad217a6a3b302166a718ba0e25920ef092fdaef3853449ecf341a1237445330",
+               "bytes_per_launch": 839.26e6 + 521.24e6}
 
 
 def log(*a):

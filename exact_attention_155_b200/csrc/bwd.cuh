@@ -691,11 +691,16 @@ __global__ void __launch_bounds__(448, 1)
       if (!ok) break;
       ++nu;
       {
-        // Epilogue: warpgroup 0 writes dV rows, warpgroup 1 writes dK rows (x scale).
+        // Epilogue: warpgroup 0 writes dV rows, warpgroup 1 writes dK rows (x scale). Each
+        // thread writes its own key row, so a warp's store touches 32 rows: 32-byte
+        // stores (when the rows allow them) halve the number of those scattered pieces,
+        // which, not the arithmetic, is what the epilogue's time goes to.
         tc_fence_after();
         const uint32_t tsrc = (half == 0 ? tDV : tDK) + lane_off;
         const float mul = half == 0 ? 1.f : p.scale;
         uint16_t* dst = (half == 0 ? p.dv + (tok0 + key) * p.rs_dv : p.dk + (tok0 + key) * p.rs_dk) + w.h * D;
+        const bool wide = (((reinterpret_cast<uintptr_t>(half == 0 ? p.dv : p.dk)) |
+                            static_cast<uintptr_t>((half == 0 ? p.rs_dv : p.rs_dk) * 2)) & 31u) == 0;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -703,13 +708,25 @@ __global__ void __launch_bounds__(448, 1)
           tmem_wait_ld();
           reg_fence32(o);
           if (key_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+            if (wide) {
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              d4[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * mul, __uint_as_float(o[8 * v + 1]) * mul),
-                                 pack_bf16x2(__uint_as_float(o[8 * v + 2]) * mul, __uint_as_float(o[8 * v + 3]) * mul),
-                                 pack_bf16x2(__uint_as_float(o[8 * v + 4]) * mul, __uint_as_float(o[8 * v + 5]) * mul),
-                                 pack_bf16x2(__uint_as_float(o[8 * v + 6]) * mul, __uint_as_float(o[8 * v + 7]) * mul));
+              for (int v = 0; v < 2; ++v) {
+                uint32_t w8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                  w8[e] = pack_bf16x2(__uint_as_float(o[16 * v + 2 * e]) * mul,
+                                      __uint_as_float(o[16 * v + 2 * e + 1]) * mul);
+                st_global_v8(dst + cc * 32 + 16 * v, w8);
+              }
+            } else {
+              uint4* d4 = reinterpret_cast<uint4*>(dst + cc * 32);
+#pragma unroll
+              for (int v = 0; v < 4; ++v)
+                d4[v] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * v]) * mul, __uint_as_float(o[8 * v + 1]) * mul),
+                                   pack_bf16x2(__uint_as_float(o[8 * v + 2]) * mul, __uint_as_float(o[8 * v + 3]) * mul),
+                                   pack_bf16x2(__uint_as_float(o[8 * v + 4]) * mul, __uint_as_float(o[8 * v + 5]) * mul),
+                                   pack_bf16x2(__uint_as_float(o[8 * v + 6]) * mul, __uint_as_float(o[8 * v + 7]) * mul));
+            }
           }
         }
       }

@@ -654,6 +654,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                                                                   : static_cast<long long>(w.b) * p.N) +
                               row_g;
         uint16_t* orow = p.out + tok * p.o_rs + w.h * D + grp * DG;
+        // Each thread writes its own row, so a warp's store touches 32 rows: one 32-byte
+        // store per 16 columns (when the rows allow it) halves those scattered pieces.
+        const bool wide = ((reinterpret_cast<uintptr_t>(p.out) | static_cast<uintptr_t>(p.o_rs * 2)) & 31u) == 0;
 #pragma unroll
         for (int cc = 0; cc < DG / 16; ++cc) {
           uint32_t o[16];
@@ -665,9 +668,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int c = 0; c < 8; ++c)
             pk[c] = pack_bf16x2(__uint_as_float(o[2 * c]) * inv_l, __uint_as_float(o[2 * c + 1]) * inv_l);
           if (row_ok) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 16);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            if (wide) {
+              st_global_v8(orow + cc * 16, pk);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(orow + cc * 16);
+              dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+              dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            }
           }
         }
         // O_t has been read: the next unit's first P V may overwrite it.

@@ -289,6 +289,15 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// ------------------------------------------------------------ global stores
+// 32 bytes from one thread (sm_100): one full sector per store instead of two halves.
+// `addr` must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* addr, const uint32_t (&v)[8]) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(addr), "r"(v[0]), "r"(v[1]),
+               "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
 // ------------------------------------------------------------------ numerics
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
