@@ -18,8 +18,9 @@
 //    pipeline fill and drain on an otherwise idle SM;
 //  * the producer warp streams K_j and V_j (128 x d bf16) through a ring of shared-memory
 //    stages with TMA (128-byte swizzle) and mbarrier full/empty pairs; the ring runs
-//    on across units, and the producer publishes each unit's index to the other roles
-//    through a small shared-memory ring;
+//    on across units, and the producer hands each unit to the other roles through a
+//    small shared-memory ring with its decoded (batch, head, row block), skipping units
+//    with nothing to do (past the end of a shorter sequence);
 //  * one MMA warp per Q tile issues tcgen05.mma from one thread: S_t = Q_t K_j^T into
 //    TMEM (fp32, 128 lanes x 128 columns per tile), then O_t += P_t V_j with P_t read
 //    straight from TMEM (bf16 packed over the first 64 columns of S_t); with two
@@ -76,7 +77,7 @@ constexpr int kFwdProducerWarp = kFwdSoftmaxWarps;
 constexpr int kFwdMmaWarp = kFwdSoftmaxWarps + 1;  // tile t: kFwdMmaWarp + t
 constexpr int kFwdThreads = 32 * (kFwdSoftmaxWarps + 3);
 static_assert(kFwdGroups == 2 || kFwdGroups == 4, "2 or 4 column groups");
-constexpr int kFwdUnitSlots = 4;  // unit indices published ahead of the consumers
+constexpr int kFwdUnitSlots = 4;  // units published ahead of the consumers
 
 template <int D>
 struct FwdLayout {
@@ -103,7 +104,9 @@ struct FwdLayout {
   static constexpr int kXMaxOff = kBarOff + kNumBars * 8;
   static constexpr int kXSumOff = kXMaxOff + 2 * kFwdGroups * 128 * 4;
   static constexpr int kMiscOff = kXSumOff + 2 * kFwdGroups * 128 * 4;
-  static constexpr int kBytes = kMiscOff + 16 + 4 * kFwdUnitSlots;
+  // kMiscOff: TMEM base, abort flag, then the unit ring: kFwdUnitSlots slots of four
+  // ints (unit index or -1 to end, batch, head, row block).
+  static constexpr int kBytes = kMiscOff + 16 + 16 * kFwdUnitSlots;
   static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
   static constexpr int kThreads = kFwdThreads;
   static constexpr uint32_t kTmemCols = 512;
@@ -129,17 +132,27 @@ struct FwdUnit {
 // few heads' K/V in L2; within a group the heaviest causal row blocks come first.
 // A unit of a variable-length batch that lies past its sequence, or whose cu_seqlens
 // entries are invalid (reported once, by the producer), has nkv_max = 0.
-template <bool CAUSAL, bool GENERAL>
-__device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, int u, bool report_bad) {
-  FwdUnit w;
+// The unit's (batch, head, 256-row block): the integer divisions of the decoding, done
+// once per unit by the producer and handed to the other roles through shared memory.
+struct FwdUnitId {
+  int b, h, qb;
+};
+__device__ __forceinline__ FwdUnitId fwd_unit_id(const FwdParams& p, int u) {
   const int G = p.head_group;
   const int per_group = G * p.num_qblocks;
   const int grp = u / per_group;
   const int rem = u % per_group;
-  const int qb = p.num_qblocks - 1 - rem / G;
   const int bh = grp * G + rem % G;
-  w.b = bh / p.H;
-  w.h = bh % p.H;
+  return FwdUnitId{bh / p.H, bh % p.H, p.num_qblocks - 1 - rem / G};
+}
+
+// The rest of the decoding, from the unit's (batch, head, row block).
+template <bool CAUSAL, bool GENERAL>
+__device__ __forceinline__ FwdUnit fwd_unit(const FwdParams& p, FwdUnitId id, bool report_bad) {
+  FwdUnit w;
+  const int qb = id.qb;
+  w.b = id.b;
+  w.h = id.h;
   w.seq0 = 0;
   w.seqlen = p.N;
   w.tb = w.b;
@@ -232,14 +245,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // Consumers read the k-th unit of this CTA from slot k % kFwdUnitSlots; -1 ends the
-  // loop. Returns false on an abort (every role then leaves its loop).
-  auto next_unit = [&](int k, int* u) -> bool {
+  // Consumers read the k-th unit of this CTA from slot k % kFwdUnitSlots (index -1 ends
+  // the loop). Returns false on an abort (every role then leaves its loop).
+  auto next_unit = [&](int k, int* u, FwdUnitId* id) -> bool {
     const int slot = k % kFwdUnitSlots;
     const bool w = __all_sync(0xffffffffu, wait_bar(BAR(L::kUnitFull + slot), (k / kFwdUnitSlots) & 1,
                                                     abort_flag, warp >= kFwdMmaWarp ? kSiteFwdMma : kSiteFwdSoftmax));
     if (!w) return false;
-    *u = unit_ring[slot];
+    const volatile int* e = unit_ring + 4 * slot;
+    *u = e[0];
+    *id = FwdUnitId{e[1], e[2], e[3]};
     __syncwarp();
     if (lane == 0) mbar_arrive(BAR(L::kUnitEmpty + slot));
     return true;
@@ -256,15 +271,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       bool ok = true;
       int u = static_cast<int>(blockIdx.x);
       for (int k = 0; ok; ++k) {
+        // Units with nothing to do (past the end of a shorter sequence) are skipped here;
+        // the other roles never see them.
+        FwdUnitId id{};
+        FwdUnit w{};
+        for (; u < p.num_units; u = static_cast<int>(gridDim.x + atomicAdd(p.ticket, 1u))) {
+          id = fwd_unit_id(p, u);
+          w = fwd_unit<CAUSAL, GENERAL>(p, id, true);
+          if (w.nkv_max > 0) break;
+        }
         // Publish unit k (or the end) once its slot has been read by every consumer.
         const int slot = k % kFwdUnitSlots;
         if (!wait_bar(BAR(L::kUnitEmpty + slot), ((k / kFwdUnitSlots) & 1) ^ 1u, abort_flag, kSiteFwdProducer))
           break;
         const bool last = u >= p.num_units;
-        unit_ring[slot] = last ? -1 : u;
+        volatile int* e = unit_ring + 4 * slot;
+        e[0] = last ? -1 : u;
+        e[1] = id.b;
+        e[2] = id.h;
+        e[3] = id.qb;
         mbar_arrive(BAR(L::kUnitFull + slot));
         if (last) break;
-        const FwdUnit w = fwd_unit<CAUSAL, GENERAL>(p, u, true);
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
           if (!ok || w.nkv[t] == 0) continue;
@@ -362,9 +389,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       for (int k = 0; ok; ++k) {
         int u = -1;
-        if (!(ok = next_unit(k, &u)) || u < 0) break;
-        const FwdUnit w = fwd_unit<CAUSAL, GENERAL>(p, u, false);
-        if (w.nkv_max == 0) continue;
+        FwdUnitId id;
+        if (!(ok = next_unit(k, &u, &id)) || u < 0) break;
+        const FwdUnit w = fwd_unit<CAUSAL, GENERAL>(p, id, false);
         const int x0 = x;  // first ring item of this unit; item x0 + 2r (+1) = K (V) of key tile J0 + r
         const int n = w.nkv[t];
         const int a = n > 0 ? w.ka[t] - w.J0 : w.nkv_max;
@@ -452,10 +479,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int u = -1;
       // The warps of a lane quarter share named barriers, so they take the same
       // decision even if an abort lands while some of them are still waiting.
-      ok = named_bar_and(kBarVote, NTQ, next_unit(k, &u));
+      FwdUnitId id;
+      ok = named_bar_and(kBarVote, NTQ, next_unit(k, &u, &id));
       if (!ok || u < 0) break;
-      const FwdUnit w = fwd_unit<CAUSAL, GENERAL>(p, u, false);
-      if (w.nkv_max == 0) continue;
+      const FwdUnit w = fwd_unit<CAUSAL, GENERAL>(p, id, false);
       const int seqlen = w.seqlen;
       float m[2] = {-INFINITY, -INFINITY};  // running row max per tile (log2 units)
       float l[2] = {0.f, 0.f};              // running exp-sum over this group's columns
