@@ -63,9 +63,25 @@ __device__ __forceinline__ void bwd_issue_ts(uint32_t d_tmem, uint32_t a_tmem, u
 
 // Converts 64 fp32 TMEM values of one row, scaled, to bf16 and stores them as 128
 // contiguous bytes (8 x 16-byte stores).
+// 64 consecutive values of one output row (a: the first 32, b: the next 32) x mul as
+// bf16. Each thread writes its own row, so a warp's store touches 32 rows: with `wide`
+// (dst 32-byte aligned) the row goes out in 32-byte pieces, half as many as 16-byte ones.
 __device__ __forceinline__ void store_row64(uint16_t* dst, const uint32_t (&a)[32],
-                                            const uint32_t (&b)[32], float mul, bool ok) {
+                                            const uint32_t (&b)[32], float mul, bool ok, bool wide) {
   if (!ok) return;
+  if (wide) {
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const uint32_t* s = v < 2 ? a : b;
+      const int o = (v & 1) * 16;
+      uint32_t w8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        w8[e] = pack_bf16x2(__uint_as_float(s[o + 2 * e]) * mul, __uint_as_float(s[o + 2 * e + 1]) * mul);
+      st_global_v8(dst + 16 * v, w8);
+    }
+    return;
+  }
   uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
   for (int v = 0; v < 8; ++v) {
@@ -76,6 +92,11 @@ __device__ __forceinline__ void store_row64(uint16_t* dst, const uint32_t (&a)[3
                        pack_bf16x2(__uint_as_float(s[o + 4]) * mul, __uint_as_float(s[o + 5]) * mul),
                        pack_bf16x2(__uint_as_float(s[o + 6]) * mul, __uint_as_float(s[o + 7]) * mul));
   }
+}
+
+// Row stores can be 32 bytes wide when the base and the row stride keep rows 32-byte aligned.
+__device__ __forceinline__ bool rows32(const uint16_t* base, long long row_stride) {
+  return ((reinterpret_cast<uintptr_t>(base) | static_cast<uintptr_t>(row_stride * 2)) & 31u) == 0;
 }
 
 // =============================================================================
@@ -396,6 +417,7 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t tsrc = (half == 0 ? tDV : tDK) + lane_off;
       const float mul = half == 0 ? 1.f : p.scale;
       uint16_t* dst = (half == 0 ? p.dv + (tok0 + key) * p.rs_dv : p.dk + (tok0 + key) * p.rs_dk) + h * D;
+      const bool wide = half == 0 ? rows32(p.dv, p.rs_dv) : rows32(p.dk, p.rs_dk);
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
         uint32_t a[32], c[32];
@@ -404,7 +426,7 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
         reg_fence32(a);
         reg_fence32(c);
-        store_row64(dst + cc * 64, a, c, mul, key_ok);
+        store_row64(dst + cc * 64, a, c, mul, key_ok, wide);
       }
     }
   }
@@ -704,6 +726,7 @@ __global__ void __launch_bounds__(320, 1)
       const uint32_t tsrc = tDQ + lane_off + half * DH;
       uint16_t* dst = p.dq + (tok0 + q) * p.rs_dq + h * D + half * DH;
       const bool row_ok = q < seqlen;
+      const bool wide = rows32(p.dq, p.rs_dq);
 #pragma unroll
       for (int cc = 0; cc < DH / 64; ++cc) {
         uint32_t a[32], c[32];
@@ -712,14 +735,24 @@ __global__ void __launch_bounds__(320, 1)
         tmem_wait_ld();
         reg_fence32(a);
         reg_fence32(c);
-        store_row64(dst + cc * 64, a, c, p.scale, row_ok);
+        store_row64(dst + cc * 64, a, c, p.scale, row_ok, wide);
       }
       if constexpr (DH == 32) {
         uint32_t a[32];
         tmem_ld32(tsrc, a);
         tmem_wait_ld();
         reg_fence32(a);
-        if (row_ok) {
+        if (row_ok && wide) {
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+            uint32_t w8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              w8[e] = pack_bf16x2(__uint_as_float(a[16 * v + 2 * e]) * p.scale,
+                                  __uint_as_float(a[16 * v + 2 * e + 1]) * p.scale);
+            st_global_v8(dst + 16 * v, w8);
+          }
+        } else if (row_ok) {
           uint4* d4 = reinterpret_cast<uint4*>(dst);
 #pragma unroll
           for (int v = 0; v < 4; ++v)
