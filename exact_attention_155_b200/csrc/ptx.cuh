@@ -32,21 +32,6 @@ __device__ __forceinline__ void report(unsigned int code, unsigned int site, uns
   }
 }
 
-// Pipeline tracing, compiled in only with -DFA_TRACE: selected threads of one CTA
-// record clock64() at pipeline events into g_trace (read back with
-// cudaMemcpyFromSymbol by a tracing build). Off by default; no cost when off.
-#ifdef FA_TRACE
-__device__ unsigned long long g_trace[1 << 16];
-#define FA_TRACE_EVENT(cond, idx)          \
-  do {                                    \
-    if (cond) fa::g_trace[(idx)] = clock64(); \
-  } while (0)
-#else
-#define FA_TRACE_EVENT(cond, idx) \
-  do {                            \
-  } while (0)
-#endif
-
 #ifndef FA_WAIT_LIMIT_CYCLES
 // About 1-2 s at B200 clocks; no legitimate wait in these kernels comes close.
 #define FA_WAIT_LIMIT_CYCLES (3000000000ll)
