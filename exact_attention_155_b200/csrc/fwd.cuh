@@ -23,7 +23,8 @@
 //    with nothing to do (past the end of a shorter sequence);
 //  * one MMA warp per Q tile issues tcgen05.mma from one thread: S_t = Q_t K_j^T into
 //    TMEM (fp32, 128 lanes x 128 columns per tile), then O_t += P_t V_j with P_t read
-//    straight from TMEM (bf16 packed over the first 64 columns of S_t); with two
+//    straight from TMEM (bf16, two keys per column: the P of keys [32g, 32g + 32) over
+//    S_t columns [32g, 32g + 16), the column group's own); with two
 //    issuing warps the tensor pipe keeps work queued while either one waits on a
 //    barrier or a commit;
 //  * the softmax warps (four groups of four, each group taking 32 of the 128 key
@@ -335,7 +336,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // ------------------------------------------------------------ MMA issuers
     // Warp kFwdMmaWarp + t issues every product of Q tile t, from one thread:
     // S_t = Q_t K_j^T into TMEM columns [128 t, 128 t + 128), then O_t += P_t V_j with
-    // P_t read back from the same columns (bf16, two keys per column), in two key
+    // P_t read back from the same columns (bf16, two keys per column; keys [32g, 32g + 32)
+    // in columns [32g, 32g + 16)), in two key
     // halves so the first half's products start while the softmax warps finish the
     // second. A ring stage is free once both warps have arrived on its empty
     // barrier: a warp that reads the stage commits after its last product on it, a
@@ -373,7 +375,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = half * 4 + k4;
           const uint64_t bd = sdesc_sw128(sKV + s * L::kTileBytes + kk * 2048, 16384, 1024);
-          umma_ts_w(tO, tS + kk * 8, bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
+          umma_ts_w(tO, tS + 32 * (kk >> 1) + 8 * (kk & 1), bd, kIdPV, (acc || kk > 0) ? 1u : 0u);
         }
       };
       auto item_wait = [&](int xi) {
@@ -529,10 +531,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           // x holds raw scores (unmasked tile) or scaled, masked scores (masked tile).
           // exps(ms): p = 2^(x*sl2 - ms) (resp. 2^(x - ms)) for this group's C columns,
           // their sum into rsum, and bf16 P (two keys per 32-bit word) into pk. store_p()
-          // writes pk to TMEM. P of keys [k, k + 32) lands in the S columns of keys
-          // [k/2, k/2 + 16), which another column group of the same rows may not have
-          // loaded yet, so P is stored only after a barrier over the row's groups: the
-          // vote (fast path) or the max exchange (exact path), both after every load.
+          // writes pk to TMEM over the first 16 of this group's own 32 S columns, which
+          // only this group has read, so P can be stored before the vote; the P V products
+          // read the four groups' P from those columns.
           float rsum = 0.f;
           uint32_t pk[C / 32][16];
           auto exps = [&](float ms) {
@@ -561,7 +562,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           auto store_p = [&]() {
             tc_fence_after();
 #pragma unroll
-            for (int ch = 0; ch < C / 32; ++ch) tmem_st16(tS + (C / 2) * grp + ch * 16, pk[ch]);
+            for (int ch = 0; ch < C / 32; ++ch) tmem_st16(tS + C * grp + ch * 16, pk[ch]);
           };
           // Fast path: exponentiate against the current reference max. If this group's
           // exponentials of every row sum to at most 256, none of them exceeds 2^8, so P
@@ -577,13 +578,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           bool exact = (i == 0) || !(sl2 >= 0.f);
           if (!exact) {
             exps(m[t]);
+            store_p();  // own columns: no other group reads them, so no need to wait for the vote
             exact = named_bar_or(kBarVote, NTQ, !w_ok || !(rsum <= 256.f));
-            if (!exact) {
-              l[t] += rsum;
-              store_p();
-            }
+            if (!exact) l[t] += rsum;
           }
           if (exact) {
+            tmem_wait_st();  // a speculative P from the fast path lands before the exact one
             // Exact path (first tile, negative scale, a grown row, or an abort): the
             // column groups exchange their maxima, move the reference, rescale O, and
             // (re)do the exponentials.
