@@ -18,7 +18,7 @@
 //    products, dK/dV epilogue and dQ reductions finish. Scores are
 //    computed transposed (keys on TMEM lanes) so P^T and dS^T are already in the
 //    A-operand orientation of dV += P^T dO and dK += dS^T Q:
-//       S^T  = K Q_i^T        (TMEM cols [0,128), fp32; P^T bf16 over [0,64))
+//       S^T  = K Q_i^T        (TMEM cols [0,128), fp32; P^T bf16 over [0,32), [64,96))
 //       dP^T = V dO_i^T       (TMEM cols [128,256), fp32)
 //       dV  += P^T dO_i       (A from TMEM, TMEM cols [256,256+d))
 //       dK  += dS^T Q_i       (A = dS^T in shared memory, TMEM [256+d,256+2d))
@@ -216,10 +216,7 @@ struct BwdLayout {
   static constexpr int kDQFree = kSFull + 6;
   static constexpr int kMmaDone = kSFull + 7;
   static constexpr int kDrain = kSFull + 8;
-  // [4] per TMEM lane quarter: the first warpgroup's warp of the quarter has loaded
-  // S^T (the second warpgroup's P^T overwrites S^T columns that warp reads).
-  static constexpr int kSLoaded = kDrain + 1;
-  static constexpr int kKVEmpty = kSLoaded + 4;      // the unit's last products read K_j, V_j
+  static constexpr int kKVEmpty = kDrain + 1;        // the unit's last products read K_j, V_j
   static constexpr int kUnitFull = kKVEmpty + 1;     // [kBwdUnitSlots]
   static constexpr int kUnitEmpty = kUnitFull + kBwdUnitSlots;  // [kBwdUnitSlots]
   static constexpr int kNumBars = kUnitEmpty + kBwdUnitSlots;
@@ -356,7 +353,6 @@ __global__ void __launch_bounds__(448, 1)
     mbar_init(BAR(L::kDQFree), 128);
     mbar_init(BAR(L::kMmaDone), 1);
     mbar_init(BAR(L::kDrain), 1);
-    for (int q = 0; q < 4; ++q) mbar_init(BAR(L::kSLoaded + q), 32);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -521,7 +517,7 @@ __global__ void __launch_bounds__(448, 1)
           tc_fence_after();
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            umma_ts_w(tDV, tS + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
+            umma_ts_w(tDV, tS + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdKV,
                     (n > 0 || kk > 0) ? 1u : 0u);
           umma_commit_w(BAR(L::kDOEmpty));
           // S^T of the next tile: the S columns are free once dV (issued above, executed
@@ -597,10 +593,6 @@ __global__ void __launch_bounds__(448, 1)
         tmem_wait_ld();
         reg_fence32(s0);
         reg_fence32(s1);
-        if (half == 0) {
-          tc_fence_before();
-          mbar_arrive(BAR(L::kSLoaded + wq));
-        }
         // Local columns c in [qlo_c, qhi_c] are the queries that see this key (window
         // [key - wr, key + wl]); none if the key is past the sequence. Queries past the
         // sequence have lse2 = +inf, so their P is already 0. Only tiles where some key of
@@ -631,17 +623,12 @@ __global__ void __launch_bounds__(448, 1)
           pk[2 * c4] = pack_bf16x2(e0, e1);
           pk[2 * c4 + 1] = pack_bf16x2(e2, e3);
         }
-        // P^T of queries [c0, c0 + 64) goes to columns [c0/2, c0/2 + 32): for the second
-        // warpgroup those are S^T columns of the first one, which must have loaded them.
-        // (The first warpgroup overwrites only its own columns; it is never more than one
-        // tile ahead, since S^T(n + 1) waits for both warpgroups' P^T(n).)
-        if (half == 1) {
-          if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kSLoaded + wq), g & 1, abort_flag,
-                                                      kSiteBwdSoftmax))))
-            break;
-        }
+        // P^T of queries [c0, c0 + 64) goes to columns [c0, c0 + 32), the first half of the
+        // S^T columns this warpgroup has just read and no other warpgroup reads, so it needs
+        // no wait. (A warpgroup is never more than one tile ahead: S^T(n + 1) waits for
+        // both warpgroups' P^T(n).)
         tc_fence_after();
-        tmem_st32(tS + lane_off + c0 / 2, pk);  // P^T bf16: two queries per 32-bit column
+        tmem_st32(tS + lane_off + c0, pk);  // P^T bf16: two queries per 32-bit column
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(BAR(L::kPFull));
