@@ -49,16 +49,18 @@ __device__ __forceinline__ void bwd_issue_ss(uint32_t d_tmem, uint32_t a, uint32
   }
 }
 // TS product accumulating into a 128 x D fp32 tile: D[tmem] (+)= A B with A a 128 x 128
-// bf16 tile in TMEM (two values per column) and B a 128 x D tile in shared memory
-// read MN-major (the contraction runs over B's 128 rows).
+// bf16 tile in TMEM and B a 128 x D tile in shared memory read MN-major (the contraction
+// runs over B's 128 rows). A's values [64h, 64h + 64) sit two per column in columns
+// [64h, 64h + 32) (h = 0, 1): each softmax warpgroup writes its half over the first half
+// of the columns it read, which the other warpgroup never reads.
 template <int D>
 __device__ __forceinline__ void bwd_issue_ts(uint32_t d_tmem, uint32_t a_tmem, uint32_t b,
                                              bool accumulate) {
   constexpr uint32_t kId = idesc_bf16_f32(128, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk)
-    umma_ts_w(d_tmem, a_tmem + kk * 8, sdesc_sw128(b + kk * 2048, 16384, 1024), kId,
-              (accumulate || kk > 0) ? 1u : 0u);
+    umma_ts_w(d_tmem, a_tmem + 64 * (kk >> 2) + 8 * (kk & 3), sdesc_sw128(b + kk * 2048, 16384, 1024),
+              kId, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // Converts 64 fp32 TMEM values of one row, scaled, to bf16 and stores them as 128
@@ -122,11 +124,7 @@ struct BwdKVLayout {
   static constexpr int kDSFull = 12;   // 256 arrivals: dS^T stored
   static constexpr int kMmaDone = 13;
   static constexpr int kDrain = 14;
-  // [4] per TMEM lane quarter: the first warpgroup's warp of the quarter has loaded
-  // S^T (resp. dP^T); the second warpgroup's P^T (dS^T) overwrites columns it reads.
-  static constexpr int kSLoaded = 15;
-  static constexpr int kDPLoaded = 19;
-  static constexpr int kNumBars = 23;
+  static constexpr int kNumBars = 15;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
   static constexpr int kThreads = 320;
@@ -196,10 +194,6 @@ __global__ void __launch_bounds__(320, 1)
     mbar_init(BAR(L::kDSFull), 256);
     mbar_init(BAR(L::kMmaDone), 1);
     mbar_init(BAR(L::kDrain), 1);
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(BAR(L::kSLoaded + q), 32);
-      mbar_init(BAR(L::kDPLoaded + q), 32);
-    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -339,10 +333,6 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
       reg_fence32(s0);
       reg_fence32(s1);
-      if (half == 0) {
-        tc_fence_before();
-        mbar_arrive(BAR(L::kSLoaded + wq));
-      }
       // Local columns c in [qlo_c, qhi_c] are the queries that see this key (window
       // [key - wr, key + wl]); none if the key is past the sequence. Queries past the
       // sequence have lse2 = +inf, so their P is already 0.
@@ -360,15 +350,10 @@ __global__ void __launch_bounds__(320, 1)
         const float p1 = (c + 1 < qlo_c || c + 1 > qhi_c) ? 0.f : e1;
         pk[c2] = pack_bf16x2(p0, p1);
       }
-      // P^T of queries [c0, c0 + 64) goes to columns [c0/2, c0/2 + 32): for the second
-      // warpgroup those are S^T columns of the first one, which must have loaded them.
-      if (half == 1) {
-        if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kSLoaded + wq), n & 1, abort_flag,
-                                                    kSiteBwdSoftmax))))
-          break;
-      }
+      // P^T of queries [c0, c0 + 64) goes to columns [c0, c0 + 32), over S^T columns this
+      // warpgroup has read and the other never reads.
       tc_fence_after();
-      tmem_st32(tS + lane_off + c0 / 2, pk);  // P^T bf16: two queries per 32-bit column
+      tmem_st32(tS + lane_off + c0, pk);  // P^T bf16: two queries per 32-bit column
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(L::kPFull));
@@ -383,10 +368,6 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
       reg_fence32(dp0);
       reg_fence32(dp1);
-      if (half == 0) {
-        tc_fence_before();
-        mbar_arrive(BAR(L::kDPLoaded + wq));
-      }
       uint32_t ds[32];
 #pragma unroll
       for (int c2 = 0; c2 < 32; ++c2) {
@@ -399,13 +380,8 @@ __global__ void __launch_bounds__(320, 1)
         ds[c2] = pack_bf16x2(d0, d1);
       }
       // dS^T goes over dP^T the same way P^T goes over S^T.
-      if (half == 1) {
-        if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDPLoaded + wq), n & 1, abort_flag,
-                                                    kSiteBwdSoftmax))))
-          break;
-      }
       tc_fence_after();
-      tmem_st32(tDP + lane_off + c0 / 2, ds);
+      tmem_st32(tDP + lane_off + c0, ds);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(L::kDSFull));
@@ -461,9 +437,8 @@ struct BwdQLayout {
   static constexpr int kSFree = kSFull + 2;          // [2] 256 arrivals: S read
   static constexpr int kDPFull = kSFull + 4;         // [2]
   static constexpr int kDSFull = kSFull + 6;         // [2] 256 arrivals: dS stored
-  static constexpr int kDPLoaded = kSFull + 8;       // [4] per lane quarter, as in dK/dV
-  static constexpr int kDQDone = kSFull + 12;
-  static constexpr int kDrain = kSFull + 13;
+  static constexpr int kDQDone = kSFull + 8;
+  static constexpr int kDrain = kSFull + 9;
   static constexpr int kNumBars = kDrain + 1;
   static constexpr int kMisc = kBar + kNumBars * 8;
   static constexpr int kBytes = kMisc + 16;
@@ -529,7 +504,6 @@ __global__ void __launch_bounds__(320, 1)
       mbar_init(BAR(L::kDPFull + t), 1);
       mbar_init(BAR(L::kDSFull + t), 256);
     }
-    for (int q = 0; q < 4; ++q) mbar_init(BAR(L::kDPLoaded + q), 32);
     mbar_init(BAR(L::kDQDone), 1);
     mbar_init(BAR(L::kDrain), 1);
     *abort_flag = 0;
@@ -691,10 +665,6 @@ __global__ void __launch_bounds__(320, 1)
       tmem_wait_ld();
       reg_fence32(dp0);
       reg_fence32(dp1);
-      if (half == 0) {
-        tc_fence_before();
-        mbar_arrive(BAR(L::kDPLoaded + wq));
-      }
       uint32_t ds[32];
 #pragma unroll
       for (int c2 = 0; c2 < 32; ++c2) {
@@ -705,15 +675,10 @@ __global__ void __launch_bounds__(320, 1)
         ds[c2] = pack_bf16x2(p0 * (__uint_as_float(dp[c & 31]) - d_r),
                              p1 * (__uint_as_float(dp[(c + 1) & 31]) - d_r));
       }
-      // dS of keys [c0, c0 + 64) goes to columns [c0/2, c0/2 + 32): for the second
-      // warpgroup those are dP columns of the first one, which must have loaded them.
-      if (half == 1) {
-        if (!(ok = __all_sync(0xffffffffu, wait_bar(BAR(L::kDPLoaded + wq), i & 1, abort_flag,
-                                                    kSiteBwdQSoftmax))))
-          break;
-      }
+      // dS of keys [c0, c0 + 64) goes to columns [c0, c0 + 32), over dP columns this
+      // warpgroup has read and the other never reads.
       tc_fence_after();
-      tmem_st32(tSP + c0 / 2, ds);
+      tmem_st32(tSP + c0, ds);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(BAR(L::kDSFull + bf));
