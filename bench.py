@@ -56,8 +56,8 @@ NOMINAL_HBM_GBS = 8000.0
 # DRAM bytes per launch of the backward main kernel from an ncu capture of the training
 # workload, valid only for the kernel source it was taken on (sha256 of csrc/bwd.cuh);
 # null otherwise.
-BWD_TRAFFIC = {"src_sha256": "9ad217a6a3b302166a718ba0e25920ef092fdaef3853449ecf341a1237445330",
-               "bytes_per_launch": 839.26e6 + 521.24e6}
+BWD_TRAFFIC = {"src_sha256": "0d3a88e3527275458e9d5b8bd589d935486a2fd3e2fc10c2e700e594ad897658",
+               "bytes_per_launch": 837.20e6 + 518.84e6}
 
 
 def log(*a):
