@@ -32,6 +32,12 @@
  *  - Ownership: the caller allocates and owns every buffer, including workspaces;
  *    the library allocates no device memory and keeps no per-call state. Inputs are
  *    read-only except the KV cache rows that fa_decode appends.
+ *  - Work scheduling: the forward and backward kernels are persistent (one CTA per
+ *    SM, each taking work units from a counter). The backward's counter lives in the
+ *    caller's workspace. The forward's comes from a pool of 64 counters in the
+ *    library's device image, one per launch in turn, zeroed on the launch's stream;
+ *    so at most 64 forward launches may be executing at the same time on one device
+ *    (more, on many streams with no ordering between them, could share a counter).
  *  - Errors: argument problems are detected on the host before anything is
  *    launched and return a non-zero status with a message from fa_last_error().
  *    Problems only visible on the device (a cache_seqlens value out of range, an
