@@ -121,7 +121,10 @@ size_t fa_bwd_workspace_size(int B, int H, int N, int d);
  *   q, k, v, out, dout : [B, N, H, d] bf16 (read);  lse : [B, H, N] fp32 (read)
  *   dq, dk, dv         : [B, N, H, d] bf16 (written)
  *   workspace          : >= fa_bwd_workspace_size(B,H,N,d) bytes, 256-byte aligned;
- *                        contents on entry are ignored and left undefined.
+ *                        contents on entry are ignored and left undefined. It holds the
+ *                        call's dQ accumulator and work-unit counter, so two calls whose
+ *                        executions may overlap (different streams, no ordering) need
+ *                        separate workspaces.
  * dq is summed over key tiles with fp32 reductions into the workspace in an order
  * that is not fixed, so dq may differ in the last bits between runs; dk and dv are
  * bitwise repeatable (fa_bwd_ex with deterministic = 1 makes dq repeatable too).
